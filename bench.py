@@ -1,0 +1,359 @@
+"""Benchmark of the B200 W4A4 linear layer (fused rotate+quantise+GEMM).
+
+Workload: the square layer M=4608 (1024^2 image latent tokens), K=3072,
+N=3072, g=128, bf16 activations with 0.5% outlier channels x30, bf16 bias; a
+step is one fused layer call (activation kernel + tensor-core GEMM) on
+inputs already resident in HBM.  Five independent input/weight/output sets
+(>2x the 126 MB L2) are rotated between steps so every step starts L2-cold.
+
+Prints one JSON line (rank 0).  ``--impl reference`` times the CPU oracle on
+a bounded sample of the same workload instead.
+"""
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+INT8_OVER_BF16 = 2.0      # nominal dense int8 : bf16 tensor throughput on B200 (4.5 : 2.25 PFLOP/s)
+N_SETS = 5
+
+
+def load_peaks():
+    if os.path.exists(PEAKS_FILE):
+        with open(PEAKS_FILE) as fh:
+            p = json.load(fh)
+        return p, "measured"
+    return FALLBACK, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling in the background."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.dev)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, ValueError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(value, world):
+    if world == 1:
+        return value
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def cpu_cores_used():
+    try:
+        from threadpoolctl import threadpool_info
+        n = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+        return int(n)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def time_oracle(cfg, rows, reps=1):
+    """Seconds per pass of the oracle layer over `rows` rows of the workload
+    (weights prepared offline, outside the timing)."""
+    import oracle as orc
+    x, W, b = cfg.make()
+    wq = orc.quantize_weight(W.numpy(), cfg.g)
+    xb = workloads.bf16_bits(x[:rows])
+    bb = workloads.bf16_bits(b) if b is not None else None
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        orc.linear(xb, wq["packed"], wq["scale"], bb, cfg.g, cfg.act)
+    return (time.perf_counter() - t0) / reps
+
+
+def run_reference(args, cfg, world, rank):
+    """The oracle, as it stands, on the host cores: each step is a bounded row
+    sample of the workload; throughput is scaled by the sampled ops."""
+    if rank != 0:
+        return
+    probe_rows = 64
+    t_probe = time_oracle(cfg, probe_rows)
+    budget = 120.0                                  # seconds of CPU for the whole run
+    per_step = budget / max(1, args.steps + args.warmup)
+    rows = int(max(8, min(cfg.M, probe_rows * per_step / max(t_probe, 1e-6))))
+    import oracle as orc
+    x, W, b = cfg.make()
+    wq = orc.quantize_weight(W.numpy(), cfg.g)
+    xb = workloads.bf16_bits(x[:rows])
+    bb = workloads.bf16_bits(b)
+    for _ in range(args.warmup):
+        orc.linear(xb, wq["packed"], wq["scale"], bb, cfg.g, cfg.act)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        orc.linear(xb, wq["packed"], wq["scale"], bb, cfg.g, cfg.act)
+    dt = (time.perf_counter() - t0) / args.steps
+    ops = 2.0 * rows * cfg.N * cfg.K
+    tops = ops / dt / 1e12
+    sample = f"{rows} of {cfg.M} rows per step (fused layer, weights prepared offline)"
+    line = {
+        "impl": "reference", "metric": "W4A4 linear TOPS (fused quant+GEMM) at M=4608",
+        "value": tops, "unit": "TOPS", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "s4xs4->s32 (f64 oracle)", "data": "synthetic",
+        "config": {"workload": cfg.name, "M": cfg.M, "K": cfg.K, "N": cfg.N, "g": cfg.g,
+                   "sampled_rows_per_step": rows},
+        "cpu_baseline": {"value": tops, "unit": "TOPS", "cores": cpu_cores_used(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": tops, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def make_sets(cfg, w4, device):
+    """N_SETS independent (x, Wq, sw, bias, y) sets, resident in HBM."""
+    sets = []
+    x0, W0, b0 = cfg.make()
+    for i in range(N_SETS):
+        if i == 0:
+            x, W, b = x0, W0, b0
+        else:
+            c = workloads.Linear(cfg.name, M=cfg.M, K=cfg.K, N=cfg.N, g=cfg.g, seed=cfg.seed + 100 * i,
+                                 outlier_frac=cfg.outlier_frac, outlier_scale=cfg.outlier_scale)
+            x, W, b = c.make()
+        xd = x.to(device)
+        Wq, sw = w4.quantize_weight(W.to(device), cfg.g)
+        bd = b.to(device)
+        y = torch.empty(cfg.M, cfg.N, dtype=torch.bfloat16, device=device)
+        Xq = torch.empty(cfg.M, cfg.K // 2, dtype=torch.int8, device=device)
+        sx = torch.empty(cfg.M, dtype=torch.float32, device=device)
+        sets.append({"x": xd, "Wq": Wq, "sw": sw, "b": bd, "y": y, "Xq": Xq, "sx": sx})
+    torch.cuda.synchronize()
+    return sets
+
+
+def time_loop(fn, steps, stream):
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    start.record(stream)
+    for i in range(steps):
+        fn(i)
+    end.record(stream)
+    end.synchronize()
+    return start.elapsed_time(end) / 1e3    # seconds
+
+
+def run_impl(args, cfg, world, rank, local):
+    import w4a4_hadamard_rotated_b200 as w4
+    w4.load_library()
+    device = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream(device)
+    sets = make_sets(cfg, w4, device)
+    g = cfg.g
+
+    def fused(i):
+        s = sets[i % N_SETS]
+        w4.linear_fused(s["x"], s["Wq"], s["sw"], s["b"], g, cfg.act, out=s["y"])
+
+    # ---- the timed region: exactly `steps` fused layer calls
+    sampler = ClockSampler(device.index) if rank == 0 else None
+    if sampler:
+        sampler.start()
+    for i in range(args.warmup):
+        fused(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    dt = time_loop(fused, args.steps, stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop() if sampler else None
+    dt_max = max_over_ranks(dt, world)
+    ops = float(cfg.ops())
+    value = world * ops * args.steps / dt_max / 1e12
+    ms_per_step = dt_max / args.steps * 1e3
+
+    # ---- per-kernel launch durations (same kernels and launch shapes, on the
+    # launching stream) for the roofline of the dominant kernel
+    def quant(i):
+        s = sets[i % N_SETS]
+        w4.quantize_activation(s["x"], g, cfg.act, out=(s["Xq"], s["sx"]))
+
+    def gemm(i):
+        s = sets[i % N_SETS]
+        w4.linear(s["Xq"], s["sx"], s["Wq"], s["sw"], s["b"], out=s["y"])
+
+    reps = max(args.steps, 20)
+    for i in range(3):
+        quant(i)
+        gemm(i)
+    t_quant = time_loop(quant, reps, stream) / reps
+    for i in range(N_SETS):
+        quant(i)
+    t_gemm = time_loop(gemm, reps, stream) / reps
+
+    # ---- end to end through the public API with host buffers: pinned x in,
+    # y out, copies inside the timed region
+    s0 = sets[0]
+    x_host = s0["x"].cpu().pin_memory()
+    y_host = torch.empty(cfg.M, cfg.N, dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(s0["x"])
+
+    def e2e(i):
+        x_dev.copy_(x_host, non_blocking=True)
+        w4.linear_fused(x_dev, s0["Wq"], s0["sw"], s0["b"], g, cfg.act, out=s0["y"])
+        y_host.copy_(s0["y"], non_blocking=True)
+
+    for i in range(3):
+        e2e(i)
+    e2e_steps = max(10, min(args.steps, 200))
+    t_e2e = time_loop(e2e, e2e_steps, stream) / e2e_steps
+    t_e2e = max_over_ranks(t_e2e, world)
+    e2e_value = world * ops / t_e2e / 1e12
+
+    err = w4.last_device_error()
+    if err != 0:
+        raise RuntimeError(f"device status {err} after the benchmark")
+
+    if rank != 0:
+        return
+    peaks, kind = load_peaks()
+    burst = peaks.get("bf16_tflops", FALLBACK["bf16_tflops"])
+    int8_peak = burst * INT8_OVER_BF16
+    gemm_tops = ops / t_gemm / 1e12
+    hbm = peaks.get("hbm_gbs", FALLBACK["hbm_gbs"])
+    quant_bytes = 2 * cfg.M * cfg.K + cfg.M * cfg.K // 2 + 4 * cfg.M
+    roof_time = max(ops / (int8_peak * 1e12), cfg.bytes() / (hbm * 1e9))
+    cpu = None
+    if world == 1 or rank == 0:
+        rows = 256
+        t_cpu = time_oracle(cfg, rows)
+        cpu = {"value": 2.0 * rows * cfg.N * cfg.K / t_cpu / 1e12, "unit": "TOPS", "cores": cpu_cores_used(),
+               "kind": "oracle", "sample": f"{rows} of {cfg.M} rows, one pass, weights prepared offline"}
+    line = {
+        "metric": "W4A4 linear TOPS (fused quant+GEMM) at M=4608",
+        "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "s4xs4->s32", "data": "synthetic",
+        "config": {"workload": cfg.name, "M": cfg.M, "K": cfg.K, "N": cfg.N, "g": cfg.g, "bias": True,
+                   "l2": f"{N_SETS} rotating input/weight/output sets (> 2x L2)",
+                   "parallelism": f"replicas x{world}"},
+        "us_per_layer": ms_per_step * 1e3,
+        "roofline_fraction_of_layer": roof_time / (ms_per_step / 1e3),
+        "layer_roofline_us": roof_time * 1e6,
+        "kernels_us": {"rotate_quant_pack": t_quant * 1e6, "gemm_tc": t_gemm * 1e6},
+        "roofline": {"bound": "tensor", "achieved": gemm_tops, "peak": int8_peak, "unit": "TOPS",
+                     "frac": gemm_tops / int8_peak, "traffic": None,
+                     "kernel": "gemm_tc (tcgen05 kind::i8)",
+                     "peak_note": f"int8 = 2 x {kind} bf16 burst {burst} TFLOP/s"},
+        "quant_kernel_roofline": {"bound": "hbm", "achieved": quant_bytes / t_quant / 1e9, "peak": hbm,
+                                  "unit": "GB/s", "frac": quant_bytes / t_quant / 1e9 / hbm},
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": "TOPS", "h2d_bytes_per_step": int(x_host.numel() * 2),
+                "d2h_bytes_per_step": int(y_host.numel() * 2)},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world, rank, local = dist_setup()
+    cfg = workloads.SQUARE
+    try:
+        if args.impl == "reference":
+            run_reference(args, cfg, world, rank)
+        else:
+            run_impl(args, cfg, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,150 @@
+/*
+ * w4a4.h -- C ABI of the B200 (sm_100a) ConvRot W4A4 linear layer.
+ *
+ * The method (page "[PR #63] int4_tensorwise: W4A4 layout (+ConvRot) with
+ * fused CUDA kernels", section "Description"):
+ *   - activations x[M,K] are rotated with a blockwise Walsh-Hadamard
+ *     transform (ConvRot; contiguous groups of g columns, natural order,
+ *     normalised by 1/sqrt(g)), then quantised per row to signed int4 with
+ *     one fp32 scale per row (scale = amax/7, round half to even, clamp to
+ *     [-7, 7]) and packed two per byte, low nibble first, into an [M, K/2]
+ *     int8 container;
+ *   - weights W[N,K] are rotated and quantised the same way once, offline,
+ *     giving packed [N, K/2] int8 plus fp32 [N] scales;
+ *   - an s4 x s4 GEMM accumulates in int32 (|acc| <= 49*K), and a rank-one
+ *     epilogue writes y[m,n] = bf16(acc * sx[m] * sw[n] + bias[n]).
+ *
+ * Conventions for every entry point:
+ *   - Every tensor pointer is DEVICE memory owned by the caller; the library
+ *     never allocates or frees memory.  Matrices are row-major with the
+ *     inner dimension contiguous; ld* arguments are row strides in elements.
+ *   - bf16 tensors are passed as raw 16-bit patterns (uint16_t).
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  All work is
+ *     enqueued asynchronously on it; the return value reports argument
+ *     checks and launch errors only.  Kernels that give up waiting record
+ *     W4A4_ERR_TIMEOUT in a device status word read by w4a4_last_device_error.
+ *   - Errors are returned as w4a4_status codes, never printed or thrown.
+ *   - Only sm_100 devices are supported (W4A4_ERR_DEVICE otherwise).
+ *   - Calls are thread-safe as long as different host threads use different
+ *     outputs and workspaces.
+ */
+#ifndef W4A4_H_
+#define W4A4_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  W4A4_OK = 0,
+  W4A4_ERR_NULL = 1,      /* a required pointer is NULL                         */
+  W4A4_ERR_SHAPE = 2,     /* a size is out of range or breaks a multiple rule   */
+  W4A4_ERR_GROUP = 3,     /* g not in {64,128,256} or does not divide K          */
+  W4A4_ERR_ALIGN = 4,     /* a pointer or leading dimension is misaligned        */
+  W4A4_ERR_WORKSPACE = 5, /* workspace missing or smaller than required          */
+  W4A4_ERR_DEVICE = 6,    /* the current device is not an sm_100 GPU             */
+  W4A4_ERR_CUDA = 7,      /* a CUDA runtime/driver call or a launch failed       */
+  W4A4_ERR_TIMEOUT = 8,   /* a kernel gave up waiting (bounded spin expired)     */
+  W4A4_ERR_ARG = 9        /* another argument is invalid (e.g. an unknown act)   */
+} w4a4_status;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* w4a4_status_string(int status);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int w4a4_version(void);
+
+/*
+ * Offline weight preparation: rotate (ConvRot) and quantise the rows of an
+ * fp32 weight.  Page "[PR #63] ...", Description: weights are "packed signed
+ * int4 pairs (low-nibble-first, [N, K/2] int8 container) with fp32 [N, 1]
+ * per-row scales".
+ *   W   [N, K] fp32, row stride ldw >= K (elements), 16-byte aligned, ldw % 4 == 0
+ *   N >= 1;  K % 128 == 0, K % g == 0, 128 <= K <= 65536;  g in {64,128,256}
+ *   Wq  [N, K/2] int8 output, contiguous rows, 16-byte aligned
+ *   sw  [N] fp32 output
+ */
+int w4a4_quantize_weight(const float* W, int64_t N, int64_t K, int64_t ldw, int g,
+                         int8_t* Wq, float* sw, void* stream);
+
+/*
+ * Run-time activation preparation (the fused "FHT rotation + rowwise int4
+ * quantize + pack in one pass" kernel of the page's Description).
+ *   x   [M, K] bf16 bits, row stride ldx >= K, 16-byte aligned, ldx % 8 == 0
+ *   act 0: none; 1: exact-erf GELU applied to x before the rotation (used to
+ *       feed an MLP down projection from the up projection's output)
+ *   Xq  [M, K/2] int8 output (contiguous rows, 16-byte aligned); sx [M] fp32
+ *   M >= 0 (M == 0 is a no-op); K and g as for w4a4_quantize_weight.
+ * A row that is all zero gets sx = 0 and all-zero codes.
+ */
+int w4a4_quantize_activation(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int g,
+                             int act, int8_t* Xq, float* sx, void* stream);
+
+/*
+ * W4A4 linear on already-quantised operands: the s4 x s4 GEMM with int32
+ * accumulation and the rank-one epilogue of the page's Description
+ * ("per-row/per-col scales factor out of the K loop").
+ *   Xq [M, K/2] int8, sx [M] fp32 (from w4a4_quantize_activation)
+ *   Wq [N, K/2] int8, sw [N] fp32 (from w4a4_quantize_weight)
+ *   bias [N] bf16 bits or NULL
+ *   y  [M, N] bf16 bits output, row stride ldy >= N, ldy % 8 == 0, 16-byte aligned
+ *   M >= 0, N >= 1, N % 8 == 0, K >= 32, K % 32 == 0; Xq/Wq 16-byte aligned
+ *   workspace: device scratch of at least w4a4_workspace_bytes(M, N, K)
+ *       bytes, 256-byte aligned (may be NULL when that size is 0).  Calls that
+ *       share one workspace must be ordered on the same stream.
+ * M <= 64 takes the weight-streaming split-K kernel, larger M the tcgen05
+ * tensor-core kernel; both give bit-identical int32 accumulators.
+ */
+int w4a4_linear(const int8_t* Xq, const float* sx, const int8_t* Wq, const float* sw,
+                const uint16_t* bias, uint16_t* y, int64_t M, int64_t N, int64_t K,
+                int64_t ldy, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Fused layer: w4a4_quantize_activation followed by w4a4_linear, with the
+ * packed activation and its scales kept in the workspace.
+ *   x [M, K] bf16 bits with row stride ldx; other arguments as above.
+ *   workspace: at least w4a4_fused_workspace_bytes(M, N, K) bytes.
+ */
+int w4a4_linear_fused(const uint16_t* x, int64_t ldx, const int8_t* Wq, const float* sw,
+                      const uint16_t* bias, uint16_t* y, int64_t ldy, int64_t M, int64_t N,
+                      int64_t K, int g, int act, void* workspace, size_t workspace_bytes,
+                      void* stream);
+
+/* Workspace sizes in bytes (0 when none is needed).  Pure host functions. */
+size_t w4a4_workspace_bytes(int64_t M, int64_t N, int64_t K);
+size_t w4a4_fused_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+/*
+ * Raw int32 accumulators acc[m, n] = sum_k qx[m,k] * qw[n,k] (no epilogue),
+ * for bit-exact checks of the GEMM.  path: 0 = tcgen05 tensor-core kernel,
+ * 1 = small-M weight-streaming kernel (M <= 64 only).
+ *   acc [M, N] int32 output with row stride ldc >= N, ldc % 4 == 0.
+ * Other rules as for w4a4_linear.
+ */
+int w4a4_gemm_s32(const int8_t* Xq, const int8_t* Wq, int32_t* acc, int64_t M, int64_t N,
+                  int64_t K, int64_t ldc, int path, void* workspace, size_t workspace_bytes,
+                  void* stream);
+
+/*
+ * Synchronise `stream`, then read and clear the device status word that
+ * kernels set when a bounded wait expires.  Returns W4A4_OK,
+ * W4A4_ERR_TIMEOUT, or W4A4_ERR_CUDA if the synchronisation failed.
+ */
+int w4a4_last_device_error(void* stream);
+
+/*
+ * Test hook for the bounded-wait machinery: launches one CTA whose only
+ * thread waits on an mbarrier that nothing ever arrives on, with a wait
+ * limit of `timeout_us` microseconds (1..1000000).  The kernel must record
+ * W4A4_ERR_TIMEOUT and return; it never traps or hangs.
+ */
+int w4a4_debug_wait_timeout(int64_t timeout_us, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* W4A4_H_ */

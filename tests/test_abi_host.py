@@ -1,0 +1,118 @@
+"""Host-only checks of the C ABI: the library loads, exports every symbol
+the header declares, and rejects invalid arguments before touching a GPU."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import w4a4_hadamard_rotated_b200 as w4
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "w4a4.h")
+
+NULL = ctypes.c_void_p(0)
+FAKE = ctypes.c_void_p(1 << 20)          # never dereferenced: every call below fails validation first
+MISALIGNED = ctypes.c_void_p((1 << 20) + 2)
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(w4a4_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return w4.load_library()
+
+
+def test_every_declared_symbol_is_exported_and_bound(lib):
+    syms = declared_symbols()
+    assert len(syms) >= 10
+    for s in syms:
+        assert hasattr(lib, s), s
+    assert set(syms) == set(w4.SIGNATURES), "binding and header disagree"
+
+
+def test_status_strings(lib):
+    for code, name in w4.STATUS_NAMES.items():
+        assert lib.w4a4_status_string(code).decode().startswith(name)
+    assert b"unknown" in lib.w4a4_status_string(99)
+    assert lib.w4a4_version() >= 100
+
+
+def test_quantize_activation_rejects_bad_arguments(lib):
+    q = lib.w4a4_quantize_activation
+    assert q(NULL, 4, 256, 256, 128, 0, FAKE, FAKE, NULL) == 1            # null x
+    assert q(FAKE, 4, 256, 256, 96, 0, FAKE, FAKE, NULL) == 3             # bad g
+    assert q(FAKE, 4, 384, 384, 256, 0, FAKE, FAKE, NULL) == 3            # g does not divide K
+    assert q(FAKE, 4, 200, 200, 64, 0, FAKE, FAKE, NULL) == 2             # K % 128
+    assert q(FAKE, 4, 256, 128, 128, 0, FAKE, FAKE, NULL) == 2            # ldx < K
+    assert q(FAKE, -1, 256, 256, 128, 0, FAKE, FAKE, NULL) == 2           # M < 0
+    assert q(FAKE, 4, 256, 256, 128, 2, FAKE, FAKE, NULL) == 9            # act
+    assert q(MISALIGNED, 4, 256, 256, 128, 0, FAKE, FAKE, NULL) == 4      # x alignment
+    assert q(FAKE, 4, 256, 260, 128, 0, FAKE, FAKE, NULL) == 4            # ldx % 8
+    assert q(FAKE, 4, 49152 + 128, 49280, 128, 0, FAKE, FAKE, NULL) == 2  # K too large
+
+
+def test_quantize_weight_rejects_bad_arguments(lib):
+    q = lib.w4a4_quantize_weight
+    assert q(FAKE, 8, 256, 256, 128, NULL, FAKE, NULL) == 1
+    assert q(FAKE, 0, 256, 256, 128, FAKE, FAKE, NULL) == 2
+    assert q(FAKE, 8, 256, 254, 128, FAKE, FAKE, NULL) == 2
+    assert q(FAKE, 8, 256, 258, 128, FAKE, FAKE, NULL) == 4
+
+
+def test_linear_rejects_bad_arguments(lib):
+    f = lib.w4a4_linear
+    args = lambda **kw: [kw.get(k, v) for k, v in (
+        ("xq", FAKE), ("sx", FAKE), ("wq", FAKE), ("sw", FAKE), ("bias", NULL), ("y", FAKE),
+        ("M", 128), ("N", 256), ("K", 256), ("ldy", 256), ("ws", NULL), ("wsb", 0), ("st", NULL))]
+    assert f(*args(xq=NULL)) == 1
+    assert f(*args(sw=NULL)) == 1
+    assert f(*args(N=12)) == 2              # N % 8
+    assert f(*args(K=48)) == 2              # K % 32
+    assert f(*args(K=0)) == 2
+    assert f(*args(M=-3)) == 2
+    assert f(*args(ldy=128)) == 2           # ldy < N
+    assert f(*args(ldy=260)) == 4           # ldy % 8
+    assert f(*args(y=MISALIGNED)) == 4
+    assert f(*args(bias=MISALIGNED)) == 4
+
+
+def test_fused_rejects_bad_arguments(lib):
+    f = lib.w4a4_linear_fused
+    base = dict(x=FAKE, ldx=256, wq=FAKE, sw=FAKE, bias=NULL, y=FAKE, ldy=256, M=100, N=256, K=256,
+                g=128, act=0, ws=NULL, wsb=0, st=NULL)
+    call = lambda **kw: f(*({**base, **kw}).values())
+    assert call(x=NULL) == 1
+    assert call(g=32) == 3
+    assert call(K=320) == 2
+    assert call(act=5) == 9
+    assert call(ldx=250) == 2
+    # every other argument is valid: the missing workspace is what fails
+    assert call() == 5
+
+
+def test_gemm_s32_rejects_bad_arguments(lib):
+    f = lib.w4a4_gemm_s32
+    assert f(FAKE, FAKE, FAKE, 128, 256, 256, 256, 2, NULL, 0, NULL) == 9      # path
+    assert f(FAKE, FAKE, FAKE, 65, 256, 256, 256, 1, NULL, 0, NULL) == 2       # small-M path, M > 64
+    assert f(FAKE, FAKE, FAKE, 16, 256, 256, 254, 0, NULL, 0, NULL) == 2       # ldc < N
+
+
+def test_workspace_sizes_are_host_functions(lib):
+    assert lib.w4a4_workspace_bytes(0, 256, 256) == 0
+    assert lib.w4a4_workspace_bytes(4608, 3072, 3072) == 0               # large M: no scratch
+    small = lib.w4a4_workspace_bytes(16, 3072, 3072)
+    assert small >= 32768 and small % 256 == 0                            # counter block + slots
+    fused = lib.w4a4_fused_workspace_bytes(4608, 3072, 3072)
+    assert fused >= 32768 + 4608 * 1536 + 4608 * 4
+    assert lib.w4a4_fused_workspace_bytes(16, 3072, 3072) >= small + 16 * 1536
+
+
+def test_debug_timeout_rejects_bad_limit(lib):
+    assert lib.w4a4_debug_wait_timeout(0, NULL) == 9
+    assert lib.w4a4_debug_wait_timeout(10_000_000, NULL) == 9

@@ -1,0 +1,254 @@
+"""GPU parity of the CUDA path against the CPU oracle, called through the C ABI
+(via the thin binding).  Sizes span several tiles and ragged tails; the full
+workloads are checked on sampled rows, which the oracle computes one by one
+(rows of the layer are independent)."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as orc
+import workloads
+from parity import (E2E_REL_L2, check_epilogue_exact, check_packed, rel_l2, to_np_bits)
+
+pytestmark = pytest.mark.gpu
+
+
+def _codes(shape, seed, lo=-7, hi=7):
+    g = torch.Generator().manual_seed(seed)
+    return torch.randint(lo, hi + 1, shape, generator=g, dtype=torch.int8).numpy()
+
+
+def _packed_cuda(q):
+    return torch.from_numpy(orc.pack_int4(q)).cuda()
+
+
+# --------------------------------------------------------------------------
+# K1: rotate + quantise + pack
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("M,K,g,act", [
+    (16, 256, 128, 0), (333, 3072, 128, 0), (333, 3072, 64, 0), (333, 3072, 256, 0),
+    (67, 12288, 128, 0), (67, 12288, 256, 1), (130, 5120, 64, 1), (1, 128, 128, 0), (5, 13824, 128, 0),
+])
+def test_quantize_activation_parity(cuda_lib, M, K, g, act):
+    x = workloads.make_activation(M, K, seed=M + K + g, outlier_frac=0.005, outlier_scale=30.0)
+    Xq, sx = cuda_lib.quantize_activation(x.cuda(), g, act)
+    ref = orc.quantize_activation(workloads.bf16_bits(x), g, act)
+    check_packed(Xq, sx, ref, f"x {M}x{K} g{g} act{act}")
+
+
+def test_quantize_activation_strided_rows(cuda_lib):
+    M, K, g = 70, 1024, 128
+    wide = workloads.make_activation(M, K + 64, seed=3, outlier_frac=0.01, outlier_scale=20.0).cuda()
+    x = wide[:, :K]
+    Xq, sx = cuda_lib.quantize_activation(x, g)
+    ref = orc.quantize_activation(workloads.bf16_bits(wide.cpu()[:, :K].contiguous()), g)
+    check_packed(Xq, sx, ref, "strided x")
+
+
+@pytest.mark.parametrize("N,K,g", [(392, 512, 128), (128, 256, 64), (200, 3072, 256), (64, 12288, 128)])
+def test_quantize_weight_parity(cuda_lib, N, K, g):
+    W = workloads.make_weight(N, K, seed=N + K)
+    Wq, sw = cuda_lib.quantize_weight(W.cuda(), g)
+    ref = orc.quantize_weight(W.numpy(), g)
+    check_packed(Wq, sw, ref, f"W {N}x{K} g{g}")
+
+
+def test_quantize_zero_rows(cuda_lib):
+    x = workloads.make_activation(40, 512, seed=9)
+    x[[0, 7, 39]] = 0
+    Xq, sx = cuda_lib.quantize_activation(x.cuda(), 128)
+    sx = sx.cpu()
+    assert sx[0] == 0 and sx[7] == 0 and sx[39] == 0
+    assert torch.all(Xq.cpu()[[0, 7, 39]] == 0)
+    check_packed(Xq, sx, orc.quantize_activation(workloads.bf16_bits(x), 128), "zero rows")
+
+
+# --------------------------------------------------------------------------
+# K2 / K3: integer GEMM, bit-exact
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("M,N,K", [(300, 392, 416), (128, 256, 128), (129, 520, 3072), (65, 8, 32),
+                                   (1000, 1032, 640), (256, 512, 12288)])
+def test_gemm_tc_exact(cuda_lib, M, N, K):
+    qa, qb = _codes((M, K), 1 + M), _codes((N, K), 2 + N)
+    acc = cuda_lib.gemm_s32(_packed_cuda(qa), _packed_cuda(qb), path=0).cpu().numpy()
+    want = orc.gemm_s32(orc.pack_int4(qa), orc.pack_int4(qb))
+    assert np.array_equal(acc, want)
+
+
+def test_gemm_tc_extremes(cuda_lib):
+    K = 12288
+    qa = np.full((130, K), 7, np.int8)
+    qa[1::2] = -7
+    qb = np.full((264, K), 7, np.int8)
+    qb[::3] = -7
+    acc = cuda_lib.gemm_s32(_packed_cuda(qa), _packed_cuda(qb), path=0).cpu().numpy()
+    assert np.array_equal(acc, orc.gemm_s32(orc.pack_int4(qa), orc.pack_int4(qb)))
+    assert np.abs(acc).max() == 49 * K
+
+
+@pytest.mark.parametrize("M", [1, 8, 16, 17, 33, 64])
+@pytest.mark.parametrize("N,K", [(392, 3072), (3072, 12288), (128, 128)])
+def test_gemm_smallm_exact(cuda_lib, M, N, K):
+    qa, qb = _codes((M, K), 5 + M), _codes((N, K), 6 + N)
+    acc = cuda_lib.gemm_s32(_packed_cuda(qa), _packed_cuda(qb), path=1).cpu().numpy()
+    want = orc.gemm_s32(orc.pack_int4(qa), orc.pack_int4(qb))
+    assert np.array_equal(acc, want)
+    # same operands through the tensor-core kernel
+    acc0 = cuda_lib.gemm_s32(_packed_cuda(qa), _packed_cuda(qb), path=0).cpu().numpy()
+    assert np.array_equal(acc0, want)
+
+
+# --------------------------------------------------------------------------
+# Rank-one epilogue and the whole layer
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("M,N,K,g,bias", [(300, 392, 512, 128, True), (16, 392, 3072, 128, True),
+                                          (64, 3072, 3072, 64, False), (513, 264, 1024, 256, False)])
+def test_linear_epilogue_exact(cuda_lib, M, N, K, g, bias):
+    x = workloads.make_activation(M, K, seed=M, outlier_frac=0.005, outlier_scale=30.0)
+    W = workloads.make_weight(N, K, seed=N)
+    b = workloads.make_bias(N, seed=N) if bias else None
+    Xq, sx = cuda_lib.quantize_activation(x.cuda(), g)
+    Wq, sw = cuda_lib.quantize_weight(W.cuda(), g)
+    y = cuda_lib.linear(Xq, sx, Wq, sw, b.cuda() if bias else None)
+    acc = orc.gemm_s32(Xq.cpu().numpy(), Wq.cpu().numpy())
+    check_epilogue_exact(y, acc, sx.cpu().numpy(), sw.cpu().numpy(),
+                         workloads.bf16_bits(b) if bias else None, f"linear {M}x{K}->{N}")
+
+
+_wq_cache = {}
+
+
+def _oracle_weight(W, g):
+    key = (tuple(W.shape), g, float(W[0, 0]), float(W[-1, -1]), float(W.sum()))
+    if key not in _wq_cache:
+        _wq_cache[key] = orc.quantize_weight(W.numpy(), g)
+    return _wq_cache[key]
+
+
+def _oracle_layer(cfg, x, W, b, rows=None):
+    """Pure-oracle layer on (a sample of) the rows."""
+    wq = _oracle_weight(W, cfg.g)
+    xb = workloads.bf16_bits(x if rows is None else x[rows])
+    return wq, orc.linear(xb, wq["packed"], wq["scale"], workloads.bf16_bits(b) if b is not None else None,
+                          cfg.g, cfg.act)
+
+
+def _check_layer(cuda_lib, cfg, x, W, b, rows=None, y=None):
+    xc, Wc = x.cuda(), W.cuda()
+    bc = b.cuda() if b is not None else None
+    Wq, sw = cuda_lib.quantize_weight(Wc, cfg.g)
+    if y is None:
+        y = cuda_lib.linear_fused(xc, Wq, sw, bc, cfg.g, cfg.act)
+    Xq, sx = cuda_lib.quantize_activation(xc, cfg.g, cfg.act)
+    wref, ref = _oracle_layer(cfg, x, W, b, rows)
+    check_packed(Wq, sw, wref, f"{cfg.name} weights")
+    sel = slice(None) if rows is None else torch.as_tensor(rows)
+    xa = orc.quantize_activation(workloads.bf16_bits(x if rows is None else x[rows]), cfg.g, cfg.act)
+    check_packed(Xq.cpu()[sel], sx.cpu()[sel], xa, f"{cfg.name} activations")
+    # the fused output equals the oracle epilogue on the GPU's own operands
+    acc = orc.gemm_s32(Xq.cpu()[sel].numpy(), Wq.cpu().numpy())
+    check_epilogue_exact(y.cpu()[sel], acc, sx.cpu()[sel].numpy(), sw.cpu().numpy(),
+                         workloads.bf16_bits(b) if b is not None else None, cfg.name)
+    err = rel_l2(to_np_bits(y.cpu()[sel]), ref["y32"])
+    assert err <= E2E_REL_L2, f"{cfg.name}: relative L2 error {err:.3g}"
+    return y
+
+
+def test_tiny_layer(cuda_lib):
+    cfg = workloads.TINY
+    x, W, b = cfg.make()
+    _check_layer(cuda_lib, cfg, x, W, b)
+
+
+@pytest.mark.parametrize("M,K,N,g", [(333, 1024, 520, 128), (130, 3072, 264, 64), (700, 2048, 1024, 256)])
+def test_medium_layers(cuda_lib, M, K, N, g):
+    cfg = workloads.Linear("medium", M=M, K=K, N=N, g=g, seed=M)
+    x, W, b = cfg.make()
+    _check_layer(cuda_lib, cfg, x, W, b)
+
+
+def _sample_rows(M, n=48, seed=0):
+    g = np.random.default_rng(seed)
+    rows = set(g.choice(M, size=n - 4, replace=False).tolist()) | {0, 1, M - 2, M - 1}
+    return sorted(rows)
+
+
+def test_square_full_size_sampled(cuda_lib):
+    cfg = workloads.SQUARE
+    x, W, b = cfg.make()
+    _check_layer(cuda_lib, cfg, x, W, b, rows=_sample_rows(cfg.M))
+
+
+def test_mlp_pair_full_size_sampled(cuda_lib):
+    up, down = workloads.MLP_UP, workloads.MLP_DOWN
+    x, Wu, bu = up.make()
+    _, Wd, bd = down.make()
+    rows = _sample_rows(up.M, 24, seed=1)
+    yu = _check_layer(cuda_lib, up, x, Wu, bu, rows=rows)
+    # the down layer reads GELU(up output), applied inside the activation kernel
+    _check_layer(cuda_lib, down, yu.cpu(), Wd, bd, rows=rows)
+
+
+@pytest.mark.parametrize("cfg", workloads.small_m_sweep(), ids=lambda c: c.name)
+def test_small_m_sweep(cuda_lib, cfg):
+    x, W, b = cfg.make()
+    _check_layer(cuda_lib, cfg, x, W, b)
+
+
+# --------------------------------------------------------------------------
+# Edge cases
+# --------------------------------------------------------------------------
+
+def test_zero_rows_give_bias(cuda_lib):
+    cfg = workloads.Linear("zero rows", M=80, K=512, N=264, g=128, seed=4)
+    x, W, b = cfg.make()
+    x[[3, 50]] = 0
+    Wq, sw = cuda_lib.quantize_weight(W.cuda(), 128)
+    y = cuda_lib.linear_fused(x.cuda(), Wq, sw, b.cuda(), 128).cpu()
+    assert torch.equal(y[3].view(torch.int16), b.view(torch.int16))
+    assert torch.equal(y[50].view(torch.int16), b.view(torch.int16))
+
+
+def test_empty_batch_is_a_no_op(cuda_lib):
+    W = workloads.make_weight(256, 512, seed=1).cuda()
+    Wq, sw = cuda_lib.quantize_weight(W, 128)
+    x = torch.empty(0, 512, dtype=torch.bfloat16, device="cuda")
+    y = cuda_lib.linear_fused(x, Wq, sw, None, 128)
+    assert y.shape == (0, 256)
+
+
+def test_repeat_calls_share_workspace_deterministically(cuda_lib):
+    # small-M split-K counters wrap back to zero, so alternating shapes on one
+    # cached workspace keep giving bit-identical results
+    outs = {}
+    for rep in range(3):
+        for (M, N, K) in ((8, 3072, 12288), (64, 392, 3072), (300, 392, 512), (16, 3072, 3072)):
+            cfg = workloads.Linear("r", M=M, K=K, N=N, g=128, seed=M)
+            x, W, b = cfg.make()
+            Wq, sw = cuda_lib.quantize_weight(W.cuda(), 128)
+            y1 = cuda_lib.linear_fused(x.cuda(), Wq, sw, b.cuda(), 128)
+            Xq, sx = cuda_lib.quantize_activation(x.cuda(), 128)
+            y2 = cuda_lib.linear(Xq, sx, Wq, sw, b.cuda())
+            assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+            key = (M, N, K)
+            if key in outs:
+                assert torch.equal(outs[key], y1.view(torch.int16))
+            outs[key] = y1.view(torch.int16).clone()
+
+
+def test_bounded_wait_reports_timeout_and_context_survives(cuda_lib):
+    lib = cuda_lib.load_library()
+    assert cuda_lib.last_device_error() == 0
+    stream = torch.cuda.current_stream().cuda_stream
+    import ctypes
+    assert lib.w4a4_debug_wait_timeout(2000, ctypes.c_void_p(stream)) == 0
+    assert cuda_lib.last_device_error() == 8          # W4A4_ERR_TIMEOUT, then cleared
+    assert cuda_lib.last_device_error() == 0
+    # the context is still usable
+    cfg = workloads.TINY
+    x, W, b = cfg.make()
+    _check_layer(cuda_lib, cfg, x, W, b)

@@ -1,0 +1,202 @@
+"""B200 (sm_100a) ConvRot W4A4 linear layer.
+
+A thin Python binding over the C ABI in ``include/w4a4.h`` (``libw4a4.so``
+next to this file).  The binding only marshals arguments: it checks tensor
+dtypes, devices and layouts, allocates outputs with PyTorch, and passes raw
+device pointers plus the current CUDA stream to the library.  Every step of
+the layer runs in the library's CUDA kernels; there is no CPU or PyTorch
+fallback, and every call raises if the library is missing or not built.
+
+Functions keep the C names without the ``w4a4_`` prefix:
+  quantize_weight(W, g)                      -> (Wq [N, K/2] int8, sw [N] fp32)
+  quantize_activation(x, g, act=0)           -> (Xq [M, K/2] int8, sx [M] fp32)
+  linear(Xq, sx, Wq, sw, bias=None)          -> y [M, N] bf16
+  linear_fused(x, Wq, sw, bias=None, g, act) -> y [M, N] bf16
+  gemm_s32(Xq, Wq, path=0)                   -> acc [M, N] int32
+"""
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libw4a4.so")
+
+OK = 0
+STATUS_NAMES = {0: "W4A4_OK", 1: "W4A4_ERR_NULL", 2: "W4A4_ERR_SHAPE", 3: "W4A4_ERR_GROUP",
+                4: "W4A4_ERR_ALIGN", 5: "W4A4_ERR_WORKSPACE", 6: "W4A4_ERR_DEVICE",
+                7: "W4A4_ERR_CUDA", 8: "W4A4_ERR_TIMEOUT", 9: "W4A4_ERR_ARG"}
+
+# Every symbol the header declares, with (restype, argtypes).
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_I = ctypes.c_int
+_SZ = ctypes.c_size_t
+SIGNATURES = {
+    "w4a4_status_string": (ctypes.c_char_p, [_I]),
+    "w4a4_version": (_I, []),
+    "w4a4_quantize_weight": (_I, [_P, _I64, _I64, _I64, _I, _P, _P, _P]),
+    "w4a4_quantize_activation": (_I, [_P, _I64, _I64, _I64, _I, _I, _P, _P, _P]),
+    "w4a4_linear": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P, _SZ, _P]),
+    "w4a4_linear_fused": (_I, [_P, _I64, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I, _I, _P, _SZ, _P]),
+    "w4a4_workspace_bytes": (_SZ, [_I64, _I64, _I64]),
+    "w4a4_fused_workspace_bytes": (_SZ, [_I64, _I64, _I64]),
+    "w4a4_gemm_s32": (_I, [_P, _P, _P, _I64, _I64, _I64, _I64, _I, _P, _SZ, _P]),
+    "w4a4_last_device_error": (_I, [_P]),
+    "w4a4_debug_wait_timeout": (_I, [_I64, _P]),
+}
+
+_lib = None
+
+
+class W4A4Error(RuntimeError):
+    def __init__(self, status, what):
+        self.status = status
+        name = STATUS_NAMES.get(status, f"status {status}")
+        super().__init__(f"{what}: {name}")
+
+
+def load_library(path=LIB_PATH):
+    """Load libw4a4.so (once) and declare its C signatures."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with __graft_entry__.build() "
+                           "(or python w4a4_hadamard_rotated_b200/build.py)")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def _check(status, what):
+    if status != OK:
+        raise W4A4Error(status, what)
+
+
+def _stream(t):
+    return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _need_cuda(t, dtype, name):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def _bits(t):
+    """View a bf16 tensor as its raw 16-bit patterns (no copy)."""
+    return t.view(torch.int16)
+
+
+# Workspaces are cached per (purpose, device, stream) and grown on demand.  The
+# small-M kernel needs its workspace zero-filled once and keeps it zero itself,
+# so the fused entry (whose workspace starts with the packed activation) gets
+# a buffer of its own.
+_workspaces = {}
+
+
+def workspace(nbytes, device, kind="linear"):
+    key = (kind, device.index if device.index is not None else torch.cuda.current_device(),
+           torch.cuda.current_stream(device).cuda_stream)
+    buf = _workspaces.get(key)
+    if buf is None or buf.numel() < nbytes:
+        buf = torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+        _workspaces[key] = buf
+    return buf
+
+
+def quantize_weight(W, g=128):
+    """Rotate + quantise fp32 weights W [N, K] -> (Wq [N, K/2] int8, sw [N] fp32)."""
+    lib = load_library()
+    _need_cuda(W, torch.float32, "W")
+    if W.dim() != 2 or W.stride(1) != 1:
+        raise ValueError("W must be a 2-D tensor with a contiguous inner dimension")
+    N, K = W.shape
+    Wq = torch.empty(N, K // 2, dtype=torch.int8, device=W.device)
+    sw = torch.empty(N, dtype=torch.float32, device=W.device)
+    _check(lib.w4a4_quantize_weight(_ptr(W), N, K, W.stride(0), g, _ptr(Wq), _ptr(sw), _stream(W)),
+           "w4a4_quantize_weight")
+    return Wq, sw
+
+
+def quantize_activation(x, g=128, act=0, out=None):
+    """Rotate + quantise bf16 activations x [M, K] -> (Xq [M, K/2] int8, sx [M] fp32)."""
+    lib = load_library()
+    _need_cuda(x, torch.bfloat16, "x")
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be a 2-D tensor with a contiguous inner dimension")
+    M, K = x.shape
+    if out is None:
+        Xq = torch.empty(M, K // 2, dtype=torch.int8, device=x.device)
+        sx = torch.empty(M, dtype=torch.float32, device=x.device)
+    else:
+        Xq, sx = out
+    _check(lib.w4a4_quantize_activation(_ptr(x), M, K, x.stride(0), g, act, _ptr(Xq), _ptr(sx), _stream(x)),
+           "w4a4_quantize_activation")
+    return Xq, sx
+
+
+def linear(Xq, sx, Wq, sw, bias=None, out=None):
+    """y [M, N] bf16 from quantised operands (int32 GEMM + rank-one epilogue)."""
+    lib = load_library()
+    _need_cuda(Xq, torch.int8, "Xq")
+    _need_cuda(Wq, torch.int8, "Wq")
+    M, Kh = Xq.shape
+    N = Wq.shape[0]
+    K = 2 * Kh
+    y = out if out is not None else torch.empty(M, N, dtype=torch.bfloat16, device=Xq.device)
+    nbytes = lib.w4a4_workspace_bytes(M, N, K)
+    ws = workspace(nbytes, Xq.device) if nbytes else None
+    _check(lib.w4a4_linear(_ptr(Xq), _ptr(sx), _ptr(Wq), _ptr(sw), _ptr(bias), _ptr(y), M, N, K, y.stride(0),
+                           _ptr(ws), nbytes, _stream(Xq)), "w4a4_linear")
+    return y
+
+
+def linear_fused(x, Wq, sw, bias=None, g=128, act=0, out=None):
+    """y [M, N] bf16 = the whole layer from bf16 activations x [M, K]."""
+    lib = load_library()
+    _need_cuda(x, torch.bfloat16, "x")
+    M, K = x.shape
+    N = Wq.shape[0]
+    y = out if out is not None else torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
+    nbytes = lib.w4a4_fused_workspace_bytes(M, N, K)
+    ws = workspace(nbytes, x.device, "fused") if nbytes else None
+    _check(lib.w4a4_linear_fused(_ptr(x), x.stride(0), _ptr(Wq), _ptr(sw), _ptr(bias), _ptr(y), y.stride(0),
+                                 M, N, K, g, act, _ptr(ws), nbytes, _stream(x)), "w4a4_linear_fused")
+    return y
+
+
+def gemm_s32(Xq, Wq, path=0, out=None):
+    """Raw int32 accumulators acc [M, N] (path 0: tcgen05 kernel, 1: small-M kernel)."""
+    lib = load_library()
+    _need_cuda(Xq, torch.int8, "Xq")
+    _need_cuda(Wq, torch.int8, "Wq")
+    M, Kh = Xq.shape
+    N = Wq.shape[0]
+    K = 2 * Kh
+    acc = out if out is not None else torch.empty(M, N, dtype=torch.int32, device=Xq.device)
+    nbytes = lib.w4a4_workspace_bytes(M, N, K) if path == 1 else 0
+    if path == 1 and nbytes == 0 and M > 0:
+        raise ValueError("path 1 (small-M kernel) needs M <= the small-M threshold")
+    ws = workspace(nbytes, Xq.device) if nbytes else None
+    _check(lib.w4a4_gemm_s32(_ptr(Xq), _ptr(Wq), _ptr(acc), M, N, K, acc.stride(0), path, _ptr(ws), nbytes,
+                             _stream(Xq)), "w4a4_gemm_s32")
+    return acc
+
+
+def last_device_error(device=None):
+    """Synchronise the current stream and return (and clear) the device status."""
+    lib = load_library()
+    dev = torch.device("cuda", torch.cuda.current_device() if device is None else device)
+    return lib.w4a4_last_device_error(ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream))

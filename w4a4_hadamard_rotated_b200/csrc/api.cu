@@ -1,0 +1,360 @@
+// C ABI of the W4A4 library: argument validation, device checks, TMA tensor
+// maps and dispatch to the kernels.  Every check that needs no GPU runs before
+// the first CUDA call, so invalid arguments are reported even on a machine
+// without a device.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstdlib>
+#include <mutex>
+
+#include "w4a4.h"
+#include "ptx.cuh"
+#include "w4a4_internal.h"
+
+namespace w4a4 {
+
+// Device status word (bounded-wait timeouts); one copy per device context.
+__device__ unsigned int g_device_status = 0;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  int checked = 0;     // 0 unknown, 1 supported, -1 unsupported
+  int num_sms = 0;
+  unsigned int* status = nullptr;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+// Resolve the current device; fills its SM count and the device address of
+// the status word on first use.
+int current_device(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return W4A4_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return W4A4_ERR_DEVICE;
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (d.checked == 0) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return W4A4_ERR_CUDA;
+    if (major != 10 || minor != 0) {
+      d.checked = -1;
+    } else {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return W4A4_ERR_CUDA;
+      d.status = static_cast<unsigned int*>(p);
+      d.num_sms = sms;
+      d.checked = 1;
+    }
+  }
+  if (d.checked < 0) return W4A4_ERR_DEVICE;
+  *out = &d;
+  return W4A4_OK;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D map over a packed int4 matrix [rows, K/2] bytes, box {64 bytes, box_rows};
+// out-of-range rows and columns read as zero.
+int packed_map(CUtensorMap* map, const int8_t* base, int64_t rows, int64_t K, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return W4A4_ERR_CUDA;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
+  const cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? W4A4_OK : W4A4_ERR_CUDA;
+}
+
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+inline size_t round256(size_t b) { return (b + 255) / 256 * 256; }
+
+int smallm_threshold() {
+  static int v = -1;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    v = kSmallMMax;
+    const char* e = std::getenv("W4A4_SMALLM_MAX");
+    if (e != nullptr) {
+      const long x = std::strtol(e, nullptr, 10);
+      if (x >= 0 && x <= kSmallMMax) v = static_cast<int>(x);
+    }
+  });
+  return v;
+}
+
+int check_quant_shape(int64_t K, int g) {
+  if (g != 64 && g != 128 && g != 256) return W4A4_ERR_GROUP;
+  if (K < 128 || K > kQuantMaxK || K % 128 != 0) return W4A4_ERR_SHAPE;
+  if (K % g != 0) return W4A4_ERR_GROUP;
+  return W4A4_OK;
+}
+
+int check_gemm_shape(int64_t M, int64_t N, int64_t K) {
+  if (M < 0 || M > (int64_t(1) << 26)) return W4A4_ERR_SHAPE;
+  if (N < 1 || N % 8 != 0 || N > (int64_t(1) << 24)) return W4A4_ERR_SHAPE;
+  if (K < 32 || K % 32 != 0 || K > (int64_t(1) << 24)) return W4A4_ERR_SHAPE;
+  return W4A4_OK;
+}
+
+
+// Shared body of w4a4_linear / w4a4_gemm_s32 after validation.
+int run_linear(const int8_t* Xq, const float* sx, const int8_t* Wq, const float* sw, const uint16_t* bias, void* out,
+               int64_t M, int64_t N, int64_t K, int64_t ldo, int out_s32, int path, void* ws, size_t ws_bytes,
+               cudaStream_t stream) {
+  DeviceInfo* dev = nullptr;
+  int st = current_device(&dev);
+  if (st != W4A4_OK) return st;
+  if (M == 0) return W4A4_OK;
+  if (path == 1) {
+    if (N > kSmallMMaxN) return W4A4_ERR_SHAPE;
+    const size_t need = smallm_workspace_bytes(M, N, K);
+    if (ws == nullptr || ws_bytes < need || !aligned(ws, 256)) return W4A4_ERR_WORKSPACE;
+    CUtensorMap tmW, tmX;
+    if ((st = packed_map(&tmW, Wq, N, K, 128)) != W4A4_OK) return st;
+    if ((st = packed_map(&tmX, Xq, M, K, smallm_rows_padded(M))) != W4A4_OK) return st;
+    SmallMArgs a{};
+    a.xq = Xq;
+    a.wq = Wq;
+    a.M = M;
+    a.N = N;
+    a.K = K;
+    a.sx = sx;
+    a.sw = sw;
+    a.bias = bias;
+    a.out = out;
+    a.ldo = ldo;
+    a.out_s32 = out_s32;
+    a.counters = static_cast<unsigned int*>(ws);
+    a.partial = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + kSmallMCounterBytes);
+    a.status = dev->status;
+    return smallm_launch_tm(tmW, tmX, a, dev->num_sms, stream) == cudaSuccess ? W4A4_OK : W4A4_ERR_CUDA;
+  }
+  CUtensorMap tmA, tmB;
+  if ((st = packed_map(&tmA, Xq, M, K, kGemmBM)) != W4A4_OK) return st;
+  if ((st = packed_map(&tmB, Wq, N, K, kGemmBN)) != W4A4_OK) return st;
+  GemmArgs a{};
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.sx = sx;
+  a.sw = sw;
+  a.bias = bias;
+  a.out = out;
+  a.ldo = ldo;
+  a.out_s32 = out_s32;
+  a.status = dev->status;
+  return gemm_tc_launch(tmA, tmB, a, dev->num_sms, stream) == cudaSuccess ? W4A4_OK : W4A4_ERR_CUDA;
+}
+
+__global__ void wait_forever_bounded_kernel(unsigned long long limit_ns, unsigned int* status) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+    // nothing ever arrives: the wait must expire and record a timeout
+    (void)mbar_wait(&bar, 0, &abort_flag, status, limit_ns);
+  }
+}
+
+}  // namespace
+}  // namespace w4a4
+
+using namespace w4a4;
+
+extern "C" {
+
+const char* w4a4_status_string(int status) {
+  switch (status) {
+    case W4A4_OK: return "W4A4_OK";
+    case W4A4_ERR_NULL: return "W4A4_ERR_NULL: a required pointer is NULL";
+    case W4A4_ERR_SHAPE: return "W4A4_ERR_SHAPE: a size is out of range or breaks a multiple rule";
+    case W4A4_ERR_GROUP: return "W4A4_ERR_GROUP: group size not in {64,128,256} or does not divide K";
+    case W4A4_ERR_ALIGN: return "W4A4_ERR_ALIGN: pointer or leading dimension misaligned";
+    case W4A4_ERR_WORKSPACE: return "W4A4_ERR_WORKSPACE: workspace missing, misaligned or too small";
+    case W4A4_ERR_DEVICE: return "W4A4_ERR_DEVICE: the current device is not an sm_100 GPU";
+    case W4A4_ERR_CUDA: return "W4A4_ERR_CUDA: a CUDA call or kernel launch failed";
+    case W4A4_ERR_TIMEOUT: return "W4A4_ERR_TIMEOUT: a kernel gave up waiting";
+    case W4A4_ERR_ARG: return "W4A4_ERR_ARG: invalid argument";
+    default: return "W4A4: unknown status";
+  }
+}
+
+int w4a4_version(void) { return 100; }
+
+int w4a4_quantize_weight(const float* W, int64_t N, int64_t K, int64_t ldw, int g, int8_t* Wq, float* sw,
+                         void* stream) {
+  if (W == nullptr || Wq == nullptr || sw == nullptr) return W4A4_ERR_NULL;
+  int st = check_quant_shape(K, g);
+  if (st != W4A4_OK) return st;
+  if (K > kQuantMaxKF32) return W4A4_ERR_SHAPE;
+  if (N < 1 || N > (int64_t(1) << 26)) return W4A4_ERR_SHAPE;
+  if (ldw < K) return W4A4_ERR_SHAPE;
+  if (ldw % 4 != 0 || !aligned(W, 16) || !aligned(Wq, 16) || !aligned(sw, 4)) return W4A4_ERR_ALIGN;
+  DeviceInfo* dev = nullptr;
+  if ((st = current_device(&dev)) != W4A4_OK) return st;
+  return rotate_quant_f32(W, N, static_cast<int>(K), ldw, g, Wq, sw, dev->num_sms, dev->status,
+                          static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? W4A4_OK
+             : W4A4_ERR_CUDA;
+}
+
+int w4a4_quantize_activation(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int g, int act, int8_t* Xq,
+                             float* sx, void* stream) {
+  if (x == nullptr || Xq == nullptr || sx == nullptr) return W4A4_ERR_NULL;
+  int st = check_quant_shape(K, g);
+  if (st != W4A4_OK) return st;
+  if (act != 0 && act != 1) return W4A4_ERR_ARG;
+  if (M < 0 || M > (int64_t(1) << 26)) return W4A4_ERR_SHAPE;
+  if (ldx < K) return W4A4_ERR_SHAPE;
+  if (ldx % 8 != 0 || !aligned(x, 16) || !aligned(Xq, 16) || !aligned(sx, 4)) return W4A4_ERR_ALIGN;
+  DeviceInfo* dev = nullptr;
+  if ((st = current_device(&dev)) != W4A4_OK) return st;
+  if (M == 0) return W4A4_OK;
+  return rotate_quant_bf16(x, M, static_cast<int>(K), ldx, g, act, Xq, sx, dev->num_sms, dev->status,
+                           static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? W4A4_OK
+             : W4A4_ERR_CUDA;
+}
+
+size_t w4a4_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  if (M <= 0 || N <= 0 || K <= 0) return 0;
+  if (M <= smallm_threshold()) return smallm_workspace_bytes(M, N, K);
+  return 0;
+}
+
+// The fused workspace always starts with the small-M counter block (even when
+// this shape takes the large-M kernel), so that the block stays at offset 0 and
+// stays zero whatever shapes share the buffer.
+static size_t fused_linear_part(int64_t M, int64_t N, int64_t K) {
+  const size_t lin = w4a4_workspace_bytes(M, N, K);
+  return round256(lin > kSmallMCounterBytes ? lin : kSmallMCounterBytes);
+}
+
+size_t w4a4_fused_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  if (M <= 0 || N <= 0 || K <= 0) return 0;
+  return fused_linear_part(M, N, K) + round256(static_cast<size_t>(M) * static_cast<size_t>(K / 2)) +
+         round256(static_cast<size_t>(M) * 4);
+}
+
+static int validate_linear(const int8_t* Xq, const float* sx, const int8_t* Wq, const float* sw,
+                           const uint16_t* bias, const void* y, int64_t M, int64_t N, int64_t K, int64_t ldy,
+                           int out_s32) {
+  if (Xq == nullptr || Wq == nullptr || y == nullptr) return W4A4_ERR_NULL;
+  if (!out_s32 && (sx == nullptr || sw == nullptr)) return W4A4_ERR_NULL;
+  int st = check_gemm_shape(M, N, K);
+  if (st != W4A4_OK) return st;
+  if (ldy < N) return W4A4_ERR_SHAPE;
+  if (!aligned(Xq, 16) || !aligned(Wq, 16) || !aligned(y, 16)) return W4A4_ERR_ALIGN;
+  if (out_s32) {
+    if (ldy % 4 != 0) return W4A4_ERR_ALIGN;
+  } else {
+    if (ldy % 8 != 0 || !aligned(sw, 16) || !aligned(sx, 4)) return W4A4_ERR_ALIGN;
+    if (bias != nullptr && !aligned(bias, 16)) return W4A4_ERR_ALIGN;
+  }
+  return W4A4_OK;
+}
+
+int w4a4_linear(const int8_t* Xq, const float* sx, const int8_t* Wq, const float* sw, const uint16_t* bias,
+                uint16_t* y, int64_t M, int64_t N, int64_t K, int64_t ldy, void* workspace, size_t workspace_bytes,
+                void* stream) {
+  int st = validate_linear(Xq, sx, Wq, sw, bias, y, M, N, K, ldy, 0);
+  if (st != W4A4_OK) return st;
+  const int path = (M <= smallm_threshold()) ? 1 : 0;
+  return run_linear(Xq, sx, Wq, sw, bias, y, M, N, K, ldy, 0, path, workspace, workspace_bytes,
+                    static_cast<cudaStream_t>(stream));
+}
+
+int w4a4_gemm_s32(const int8_t* Xq, const int8_t* Wq, int32_t* acc, int64_t M, int64_t N, int64_t K, int64_t ldc,
+                  int path, void* workspace, size_t workspace_bytes, void* stream) {
+  int st = validate_linear(Xq, nullptr, Wq, nullptr, nullptr, acc, M, N, K, ldc, 1);
+  if (st != W4A4_OK) return st;
+  if (path != 0 && path != 1) return W4A4_ERR_ARG;
+  if (path == 1 && M > kSmallMMax) return W4A4_ERR_SHAPE;
+  return run_linear(Xq, nullptr, Wq, nullptr, nullptr, acc, M, N, K, ldc, 1, path, workspace, workspace_bytes,
+                    static_cast<cudaStream_t>(stream));
+}
+
+int w4a4_linear_fused(const uint16_t* x, int64_t ldx, const int8_t* Wq, const float* sw, const uint16_t* bias,
+                      uint16_t* y, int64_t ldy, int64_t M, int64_t N, int64_t K, int g, int act, void* workspace,
+                      size_t workspace_bytes, void* stream) {
+  if (x == nullptr || Wq == nullptr || sw == nullptr || y == nullptr) return W4A4_ERR_NULL;
+  int st = check_quant_shape(K, g);
+  if (st != W4A4_OK) return st;
+  if (act != 0 && act != 1) return W4A4_ERR_ARG;
+  if ((st = check_gemm_shape(M, N, K)) != W4A4_OK) return st;
+  if (ldx < K || ldy < N) return W4A4_ERR_SHAPE;
+  if (ldx % 8 != 0 || !aligned(x, 16)) return W4A4_ERR_ALIGN;
+  if (ldy % 8 != 0 || !aligned(y, 16) || !aligned(Wq, 16) || !aligned(sw, 16)) return W4A4_ERR_ALIGN;
+  if (bias != nullptr && !aligned(bias, 16)) return W4A4_ERR_ALIGN;
+  if (M == 0) {
+    DeviceInfo* dev = nullptr;
+    return current_device(&dev);
+  }
+  const size_t need = w4a4_fused_workspace_bytes(M, N, K);
+  if (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 256)) return W4A4_ERR_WORKSPACE;
+  // Layout: [linear workspace, counter block first][packed x][sx], so that the
+  // counter block sits at offset 0 for every shape and every entry point.
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const size_t lin_bytes = fused_linear_part(M, N, K);
+  int8_t* xq = reinterpret_cast<int8_t*>(ws + lin_bytes);
+  float* sx = reinterpret_cast<float*>(ws + lin_bytes + round256(static_cast<size_t>(M) * static_cast<size_t>(K / 2)));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((st = w4a4_quantize_activation(x, M, K, ldx, g, act, xq, sx, stream)) != W4A4_OK) return st;
+  const int path = (M <= smallm_threshold()) ? 1 : 0;
+  return run_linear(xq, sx, Wq, sw, bias, y, M, N, K, ldy, 0, path, ws, lin_bytes, s);
+}
+
+int w4a4_last_device_error(void* stream) {
+  DeviceInfo* dev = nullptr;
+  int st = current_device(&dev);
+  if (st != W4A4_OK) return st;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return W4A4_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpy(&v, dev->status, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return W4A4_ERR_CUDA;
+  if (v != 0) {
+    const unsigned int zero = 0;
+    if (cudaMemcpy(dev->status, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return W4A4_ERR_CUDA;
+    return W4A4_ERR_TIMEOUT;
+  }
+  return W4A4_OK;
+}
+
+int w4a4_debug_wait_timeout(int64_t timeout_us, void* stream) {
+  if (timeout_us < 1 || timeout_us > 1000000) return W4A4_ERR_ARG;
+  DeviceInfo* dev = nullptr;
+  int st = current_device(&dev);
+  if (st != W4A4_OK) return st;
+  wait_forever_bounded_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<unsigned long long>(timeout_us) * 1000ull, dev->status);
+  return cudaGetLastError() == cudaSuccess ? W4A4_OK : W4A4_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,68 @@
+// Internal launch interfaces shared by the kernel files and the C-ABI layer.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+namespace w4a4 {
+
+// ---- activation / weight rotate + quantise + pack (quant.cu)
+cudaError_t rotate_quant_bf16(const uint16_t* x, int64_t M, int K, int64_t ldx, int g, int act, int8_t* out,
+                              float* scale, int num_sms, unsigned int* status, cudaStream_t stream);
+cudaError_t rotate_quant_f32(const float* x, int64_t M, int K, int64_t ldx, int g, int8_t* out, float* scale,
+                             int num_sms, unsigned int* status, cudaStream_t stream);
+// Largest K the in-register rotate kernel supports: 384 threads x 128 codes
+// for bf16 rows, 192 threads x 128 codes for fp32 rows (weights).
+constexpr int kQuantMaxK = 384 * 128;
+constexpr int kQuantMaxKF32 = 192 * 128;
+
+// ---- tcgen05 GEMM (gemm.cu)
+struct GemmArgs {
+  int64_t M, N, K;        // K in int4 elements
+  const float* sx;        // [M]
+  const float* sw;        // [N]
+  const uint16_t* bias;   // [N] bf16 bits or nullptr
+  void* out;              // bf16 bits [M, ldo] or int32 [M, ldo]
+  int64_t ldo;
+  int out_s32;            // 1: raw int32 accumulators
+  unsigned int* status;   // device status word (bounded-wait timeouts)
+};
+// tmA: packed activations [M, K/2] bytes, box {64, 128}; tmB: packed weights
+// [N, K/2] bytes, box {64, 256}.
+cudaError_t gemm_tc_launch(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a, int num_sms,
+                           cudaStream_t stream);
+constexpr int kGemmBM = 128;
+constexpr int kGemmBN = 256;
+
+// ---- small-M weight-streaming GEMM (smallm.cu)
+struct SmallMArgs {
+  const int8_t* xq;       // [M, K/2]
+  const int8_t* wq;       // [N, K/2]
+  int64_t M, N, K;
+  const float* sx;
+  const float* sw;
+  const uint16_t* bias;
+  void* out;
+  int64_t ldo;
+  int out_s32;
+  int32_t* partial;       // workspace: [splits, M, N] int32 split-K partial tiles
+  unsigned int* counters; // workspace: one arrival counter per N tile (zero between calls)
+  unsigned int* status;   // device status word
+};
+// tmW: packed weights [N, K/2] bytes, box {64, 128}; tmX: packed activations
+// [M, K/2] bytes, box {64, smallm_rows_padded(M)}.
+cudaError_t smallm_launch_tm(const CUtensorMap& tmW, const CUtensorMap& tmX, const SmallMArgs& a, int num_sms,
+                             cudaStream_t stream);
+int smallm_rows_padded(int64_t M);
+size_t smallm_workspace_bytes(int64_t M, int64_t N, int64_t K);
+constexpr int kSmallMMax = 64;
+// Every workspace starts with a block of arrival counters (one per 128-row
+// weight tile, so N <= 8192 * 128) that must be zero before the first call
+// and is left zero by every call.
+constexpr size_t kSmallMCounterBytes = 32768;
+constexpr int64_t kSmallMMaxN = static_cast<int64_t>(kSmallMCounterBytes / 4) * 128;
+
+}  // namespace w4a4
