@@ -118,7 +118,8 @@ int check_quant_shape(int64_t K, int g) {
 int check_gemm_shape(int64_t M, int64_t N, int64_t K) {
   if (M < 0 || M > (int64_t(1) << 26)) return W4A4_ERR_SHAPE;
   if (N < 1 || N % 8 != 0 || N > (int64_t(1) << 24)) return W4A4_ERR_SHAPE;
-  if (K < 32 || K % 32 != 0 || K > (int64_t(1) << 24)) return W4A4_ERR_SHAPE;
+  // K <= 2^17 keeps the widened accumulator 256*acc (|.| <= 12544*K) in int32
+  if (K < 32 || K % 32 != 0 || K > (int64_t(1) << 17)) return W4A4_ERR_SHAPE;
   return W4A4_OK;
 }
 
@@ -155,9 +156,6 @@ int run_linear(const int8_t* Xq, const float* sx, const int8_t* Wq, const float*
     a.status = dev->status;
     return smallm_launch_tm(tmW, tmX, a, dev->num_sms, stream) == cudaSuccess ? W4A4_OK : W4A4_ERR_CUDA;
   }
-  CUtensorMap tmA, tmB;
-  if ((st = packed_map(&tmA, Xq, M, K, kGemmBM)) != W4A4_OK) return st;
-  if ((st = packed_map(&tmB, Wq, N, K, kGemmBN)) != W4A4_OK) return st;
   GemmArgs a{};
   a.M = M;
   a.N = N;
@@ -169,7 +167,7 @@ int run_linear(const int8_t* Xq, const float* sx, const int8_t* Wq, const float*
   a.ldo = ldo;
   a.out_s32 = out_s32;
   a.status = dev->status;
-  return gemm_tc_launch(tmA, tmB, a, dev->num_sms, stream) == cudaSuccess ? W4A4_OK : W4A4_ERR_CUDA;
+  return gemm_tc_launch(Xq, Wq, a, dev->num_sms, stream) == cudaSuccess ? W4A4_OK : W4A4_ERR_CUDA;
 }
 
 __global__ void wait_forever_bounded_kernel(unsigned long long limit_ns, unsigned int* status) {
@@ -228,7 +226,8 @@ int w4a4_quantize_weight(const float* W, int64_t N, int64_t K, int64_t ldw, int 
 
 int w4a4_quantize_activation(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int g, int act, int8_t* Xq,
                              float* sx, void* stream) {
-  if (x == nullptr || Xq == nullptr || sx == nullptr) return W4A4_ERR_NULL;
+  // an empty batch (M == 0) may pass NULL for its zero-size tensors
+  if (M != 0 && (x == nullptr || Xq == nullptr || sx == nullptr)) return W4A4_ERR_NULL;
   int st = check_quant_shape(K, g);
   if (st != W4A4_OK) return st;
   if (act != 0 && act != 1) return W4A4_ERR_ARG;
@@ -267,8 +266,9 @@ size_t w4a4_fused_workspace_bytes(int64_t M, int64_t N, int64_t K) {
 static int validate_linear(const int8_t* Xq, const float* sx, const int8_t* Wq, const float* sw,
                            const uint16_t* bias, const void* y, int64_t M, int64_t N, int64_t K, int64_t ldy,
                            int out_s32) {
-  if (Xq == nullptr || Wq == nullptr || y == nullptr) return W4A4_ERR_NULL;
-  if (!out_s32 && (sx == nullptr || sw == nullptr)) return W4A4_ERR_NULL;
+  if (Wq == nullptr || (!out_s32 && sw == nullptr)) return W4A4_ERR_NULL;
+  // an empty batch (M == 0) may pass NULL for its zero-size tensors
+  if (M != 0 && (Xq == nullptr || y == nullptr || (!out_s32 && sx == nullptr))) return W4A4_ERR_NULL;
   int st = check_gemm_shape(M, N, K);
   if (st != W4A4_OK) return st;
   if (ldy < N) return W4A4_ERR_SHAPE;
@@ -305,7 +305,9 @@ int w4a4_gemm_s32(const int8_t* Xq, const int8_t* Wq, int32_t* acc, int64_t M, i
 int w4a4_linear_fused(const uint16_t* x, int64_t ldx, const int8_t* Wq, const float* sw, const uint16_t* bias,
                       uint16_t* y, int64_t ldy, int64_t M, int64_t N, int64_t K, int g, int act, void* workspace,
                       size_t workspace_bytes, void* stream) {
-  if (x == nullptr || Wq == nullptr || sw == nullptr || y == nullptr) return W4A4_ERR_NULL;
+  if (Wq == nullptr || sw == nullptr) return W4A4_ERR_NULL;
+  // an empty batch (M == 0) may pass NULL for its zero-size tensors
+  if (M != 0 && (x == nullptr || y == nullptr)) return W4A4_ERR_NULL;
   int st = check_quant_shape(K, g);
   if (st != W4A4_OK) return st;
   if (act != 0 && act != 1) return W4A4_ERR_ARG;

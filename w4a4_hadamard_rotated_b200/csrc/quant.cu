@@ -3,26 +3,38 @@
 // kernels", Description: "FHT rotation ... + rowwise int4 quantize + pack in
 // one pass").  The same kernel, with fp32 input, prepares the weights offline.
 //
-// B200 design
-//   * A CTA owns a tile of P rows.  Every row is split into S = K/128 slabs of
-//     128 consecutive elements and each thread owns one slab, entirely in
-//     registers: the Walsh-Hadamard butterflies of a group (g = 64 or 128) run
-//     on registers with no shuffles; g = 256 spans two slabs held by adjacent
-//     lanes and takes one shuffle stage.
-//   * Rows reach shared memory through bulk-async (TMA) copies into a double
-//     buffer, so the copy of the next tile overlaps the arithmetic of this one.
-//   * A lane reads its slab in XOR-swizzled 16-byte chunks (chunk j from
-//     position j ^ L, L = lane & 7), which keeps the 128-bit shared loads free
-//     of bank conflicts.  Permuting the input of a Walsh-Hadamard transform by
-//     an XOR of the index only flips signs of the output: H(x[. ^ a])[i] =
-//     (-1)^popcount(i & a) H(x)[i].  The sign of each output chunk is folded
-//     into the quantisation multiplier, and since the quantiser is odd
-//     (round-half-even and the clamp are symmetric) the codes are exact.
-//   * The row amax is reduced with shared-memory atomics on the float bits,
-//     then each thread quantises its slab (RNE of r / s with s = amax / 7,
-//     taken in fp32 exactly as r / s: a reciprocal multiply is used away from
-//     rounding boundaries and an exact division near them), packs 8 nibbles per
-//     32-bit word low nibble first and writes 64 bytes with 128-bit stores.
+// B200 design (an HBM-bound pass that is close to ALU-bound as well: 2 bytes
+// read, half a byte written, ~log2(g) adds per code)
+//   * Every row is split into S = K/128 slabs of 128 consecutive elements and
+//     each thread owns one slab, entirely in registers, as 64 packed fp32
+//     pairs (element i, element i + 64).  Six radix-2 Walsh-Hadamard stages run
+//     as paired sm_100 add/sub.f32x2 instructions (two lanes per instruction),
+//     the seventh (distance 64, g >= 128) pairs the two halves of a register;
+//     g = 256 spans two slabs held by adjacent lanes and takes one shuffle
+//     stage.
+//   * The kernel is persistent: a CTA walks row tiles (P whole rows) with a
+//     grid stride, and one thread streams the rows of the coming tiles into a
+//     3-4 deep shared-memory ring with bulk-async (TMA) copies, so HBM reads
+//     stay in flight during the arithmetic and every SM gets the same, fully
+//     coalesced request pattern.  The one CTA barrier per tile (for the row
+//     amax) also frees the ring slot that tile used.
+//   * A lane reads its slab from shared memory in XOR-swizzled 16-byte chunks
+//     (chunk j from position j ^ L, L = lane & 7), which keeps the 128-bit
+//     shared loads free of bank conflicts.  Permuting the input of a Walsh-Hadamard
+//     transform by an XOR of the index only flips signs of the output:
+//     H(x[. ^ a])[i] = (-1)^popcount(i & a) H(x)[i].  The sign of each output
+//     chunk is folded into the quantisation multiplier; the quantiser is odd
+//     (round-half-even and the clamp are symmetric), so the codes are exact.
+//   * The row amax is reduced with shared-memory atomics on the float bits
+//     (triple-buffered slots, one barrier per tile).  The code is round-half-
+//     even of r / s with s = amax / 7, taken in fp32: a reciprocal multiply
+//     and a magic-number rounding put the code in the low mantissa bits, a
+//     Horner chain of integer multiply-adds packs 8 codes per word, and if any
+//     element of the slab lies within 4e-6 of a rounding boundary those codes
+//     are decided again exactly (an fp64 comparison, see exact_code), so the
+//     codes equal those of the fp32 quotient r / s.
+//   * Codes are stored low nibble first, 64 contiguous bytes per thread, with
+//     128-bit stores.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -33,226 +45,357 @@
 
 namespace w4a4 {
 
-constexpr int kSlab = 128;  // elements per thread
+constexpr int kSlab = 128;     // elements per thread
+constexpr int kHalf = 64;      // packed pairs per thread
+constexpr int kMaxRows = 64;   // rows per CTA tile
 
 template <typename TIn>
 struct InTraits;
 template <>
 struct InTraits<uint16_t> {  // bf16 bits
   static constexpr int kChunkElems = 8;
-  static constexpr int kMaxThreads = 384;
+  static constexpr int kMaxThreads = 256;
 };
 template <>
-struct InTraits<float> {
+struct InTraits<float> {     // fp32 weights (offline)
   static constexpr int kChunkElems = 4;
   static constexpr int kMaxThreads = 192;
 };
+constexpr int kMaxStages = 4;
+constexpr size_t kRingBytes = 200 * 1024;   // shared memory for the row ring
+
+// ---- packed fp32 pairs (sm_100 .f32x2 arithmetic)
+__device__ __forceinline__ uint64_t pk2(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void upk2(uint64_t r, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
 
 __device__ __forceinline__ float gelu_erf(float t) {
   return 0.5f * t * (1.0f + erff(t * 0.70710678118654752f));
 }
 
-// Load one 16-byte chunk of the slab into 8 (bf16) or 4 (fp32) floats.
-__device__ __forceinline__ void load_chunk(const uint16_t* src, float* dst) {
-  const uint4 w = *reinterpret_cast<const uint4*>(src);
-  const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+// Element e of a 16-byte chunk as fp32.
+__device__ __forceinline__ float elem(const uint4 w, int e, const uint16_t*) {
+  const uint32_t word = e < 2 ? w.x : (e < 4 ? w.y : (e < 6 ? w.z : w.w));
+  return (e & 1) ? __uint_as_float(word & 0xFFFF0000u) : __uint_as_float(word << 16);
+}
+__device__ __forceinline__ float elem(const uint4 w, int e, const float*) {
+  return __uint_as_float(e == 0 ? w.x : (e == 1 ? w.y : (e == 2 ? w.z : w.w)));
+}
+
+// One radix-2 butterfly stage at distance H (< 64) over the packed pairs.
+template <int H>
+__device__ __forceinline__ void fht_stage2(uint64_t (&V)[kHalf]) {
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    dst[2 * i] = __uint_as_float(ws[i] << 16);
-    dst[2 * i + 1] = __uint_as_float(ws[i] & 0xFFFF0000u);
+  for (int i0 = 0; i0 < kHalf; i0 += 2 * H) {
+#pragma unroll
+    for (int i = 0; i < H; ++i) {
+      const uint64_t a = V[i0 + i], c = V[i0 + i + H];
+      V[i0 + i] = add2(a, c);
+      V[i0 + i + H] = sub2(a, c);
+    }
   }
 }
-__device__ __forceinline__ void load_chunk(const float* src, float* dst) {
-  const float4 w = *reinterpret_cast<const float4*>(src);
-  dst[0] = w.x;
-  dst[1] = w.y;
-  dst[2] = w.z;
-  dst[3] = w.w;
+
+// The code of one element taken exactly as the method states it, without a
+// division: r = fl(u * norm), and the code is round-half-even of the fp32
+// quotient fl(r / s).  `q` is a fast estimate of r / s that lies within 4e-6
+// of the boundary b = k + 1/2.  fl(r / s) equals b exactly when |r/s - b| is at
+// most half an fp32 ulp of b (b's own mantissa is even, so the ties at the
+// ends go to b); otherwise it lies strictly on one side.  Both tests are
+// exact in fp64: b has at most 5 significant bits, so b*s is exact; r and b*s
+// are within a factor of 2, so their difference is exact (Sterbenz); and the
+// half ulp is a power of two.
+__device__ __forceinline__ uint32_t exact_code(float u, float norm, float sc, float q) {
+  const float r = __fmul_rn(u, norm);
+  const float b = floorf(q) + 0.5f;
+  const double d = static_cast<double>(r) - static_cast<double>(b) * static_cast<double>(sc);
+  const float half_ulp = __int_as_float((((__float_as_int(b) >> 23) & 0xFF) - 24) << 23);
+  const double t = static_cast<double>(half_ulp) * static_cast<double>(sc);
+  const float k = d > t ? ceilf(b) : (d < -t ? floorf(b) : rintf(b));
+  return static_cast<uint32_t>(static_cast<int>(k)) & 0xFu;
 }
+
+// 1.5 * 2^23 + 8: adding it to |q| <= 7.5 rounds q to an integer k, half to
+// even, and leaves k + 8 (in 1..15) in the low four bits of the sum.
+constexpr float kMagic8 = 12582920.0f;
+constexpr uint32_t kMagicBits = 0x4B400000u;   // bits of 1.5 * 2^23
+// Horner-packing eight sums (kMagicBits + n_e) as sum_e bits_e * 16^e leaves
+// this constant on top of the nibbles n_e (mod 2^32).
+constexpr uint32_t kHornerBias = kMagicBits * 0x11111111u;
+// Near-boundary test: (q - k)^2 - (0.5 - 4e-6)^2 >= 0.
+constexpr float kNearSq = (0.5f - 4e-6f) * (0.5f - 4e-6f);
 
 template <typename TIn, int G, int ACT>
 __global__ void __launch_bounds__(InTraits<TIn>::kMaxThreads, 1)
     rotate_quant_pack_kernel(const TIn* __restrict__ x, int64_t M, int K, int64_t ldx, int rows_per_tile,
-                             int8_t* __restrict__ out, float* __restrict__ scale,
+                             int nstages, int8_t* __restrict__ out, float* __restrict__ scale,
                              unsigned int* status) {
   constexpr int C = InTraits<TIn>::kChunkElems;
-  constexpr int NCH = kSlab / C;  // chunks per slab
-  constexpr int GS = G < kSlab ? G : kSlab;  // group span inside one slab
+  constexpr int NCH = kSlab / C;   // 16-byte chunks per slab
 
-  extern __shared__ __align__(128) uint8_t smem_raw[];
-  __shared__ uint64_t full_bar[2];
-  __shared__ unsigned int row_amax[2][64];
+  extern __shared__ __align__(128) uint8_t ring[];
+  __shared__ uint64_t full[kMaxStages];
+  __shared__ unsigned int row_amax[3][kMaxRows];
   __shared__ int abort_flag;
 
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int S = K / kSlab;
   const int P = rows_per_tile;
-  const int64_t ntiles = (M + P - 1) / P;
-  const size_t row_bytes = static_cast<size_t>(K) * sizeof(TIn);
-  TIn* buf[2] = {reinterpret_cast<TIn*>(smem_raw), reinterpret_cast<TIn*>(smem_raw + P * row_bytes)};
-
-  if (tid == 0) {
-    mbar_init(&full_bar[0], 1);
-    mbar_init(&full_bar[1], 1);
-    abort_flag = 0;
-    fence_mbar_init();
-  }
-  for (int i = tid; i < 2 * 64; i += blockDim.x) (&row_amax[0][0])[i] = 0u;
-  __syncthreads();
-
-  auto issue = [&](int64_t tile, int b) {
-    const int64_t r0 = tile * P;
-    const int rows = static_cast<int>(M - r0 < P ? M - r0 : P);
-    mbar_arrive_expect_tx(&full_bar[b], static_cast<uint32_t>(rows * row_bytes));
-    if (ldx == K) {
-      bulk_load(buf[b], x + r0 * ldx, static_cast<uint32_t>(rows * row_bytes), &full_bar[b]);
-    } else {
-      for (int r = 0; r < rows; ++r)
-        bulk_load(reinterpret_cast<uint8_t*>(buf[b]) + r * row_bytes, x + (r0 + r) * ldx,
-                  static_cast<uint32_t>(row_bytes), &full_bar[b]);
-    }
-  };
-
-  if (tid == 0 && blockIdx.x < ntiles) issue(blockIdx.x, 0);
-
   const int p = tid / S;       // row inside the tile
   const int s = tid - p * S;   // slab inside the row
   const bool active = p < P;
   const int L = lane & 7;      // chunk swizzle of this lane
   const float norm = G == 64 ? 0.125f : (G == 256 ? 0.0625f : 0.0883883476483184405f);
+  const int64_t ntiles = (M + P - 1) / P;
+  const size_t row_bytes = static_cast<size_t>(K) * sizeof(TIn);
+  const size_t stage_bytes = static_cast<size_t>(P) * row_bytes;
+
+  for (int i = tid; i < 3 * kMaxRows; i += blockDim.x) (&row_amax[0][0])[i] = 0u;
+  if (tid == 0) {
+    for (int i = 0; i < kMaxStages; ++i) mbar_init(&full[i], 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  // Thread 0 streams tile `tl` into ring slot `st`.
+  auto issue = [&](int64_t tl, int st) {
+    const int64_t r0 = tl * P;
+    const int rows = static_cast<int>(M - r0 < P ? M - r0 : P);
+    uint8_t* dst = ring + st * stage_bytes;
+    mbar_arrive_expect_tx(&full[st], static_cast<uint32_t>(rows * row_bytes));
+    if (ldx == K) {
+      bulk_load(dst, x + r0 * ldx, static_cast<uint32_t>(rows * row_bytes), &full[st]);
+    } else {
+      for (int r = 0; r < rows; ++r)
+        bulk_load(dst + r * row_bytes, x + (r0 + r) * ldx, static_cast<uint32_t>(row_bytes), &full[st]);
+    }
+  };
+  int64_t issued = 0;   // copies thread 0 has issued (counts only in thread 0)
+  if (tid == 0) {
+    for (int i = 0; i < nstages; ++i) {
+      const int64_t tl = blockIdx.x + static_cast<int64_t>(i) * gridDim.x;
+      if (tl < ntiles) {
+        issue(tl, i);
+        ++issued;
+      }
+    }
+  }
 
   int it = 0;
   for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
-    const int b = it & 1;
-    const int64_t next = tile + gridDim.x;
-    if (tid == 0 && next < ntiles) issue(next, b ^ 1);
-
+    const int st = it % nstages;
     const int64_t row = tile * P + p;
-    const bool valid = active && row < M;
-    // Every thread waits (bounded) so that no copy is in flight into a buffer
-    // that the CTA has stopped tracking.
-    const bool ok = mbar_wait(&full_bar[b], (it >> 1) & 1, &abort_flag, status);
+    const bool ok = warp_wait(&full[st], static_cast<uint32_t>((it / nstages) & 1), &abort_flag, status);
+    const bool valid = active && row < M && ok;
 
-    float v[kSlab];
-    float amax = 0.0f;
-    if (valid && ok) {
-      const TIn* src = buf[b] + static_cast<size_t>(p) * K + static_cast<size_t>(s) * kSlab;
+    // Slot chunk j (j < NCH/2) fills the low halves of V[C*j .. C*j+C), slot
+    // chunk j + NCH/2 the high halves: V[i] = (element i, element i + 64).
+    uint64_t V[kHalf];
+    {
+      const uint8_t* src = ring + st * stage_bytes + p * row_bytes + static_cast<size_t>(s) * kSlab * sizeof(TIn);
 #pragma unroll
-      for (int j = 0; j < NCH; ++j) load_chunk(src + ((j ^ L) * C), &v[j * C]);
-      if (ACT == 1) {
-#pragma unroll
-        for (int i = 0; i < kSlab; ++i) v[i] = gelu_erf(v[i]);
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < kSlab; ++i) v[i] = 0.0f;
-    }
-    // Radix-2 Walsh-Hadamard butterflies inside each group of the slab (all
-    // lanes run them, so the g = 256 shuffle stage below stays convergent).
-#pragma unroll
-    for (int h = 1; h < GS; h <<= 1) {
-#pragma unroll
-      for (int i0 = 0; i0 < kSlab; i0 += 2 * h) {
-#pragma unroll
-        for (int i = i0; i < i0 + h; ++i) {
-          const float a = v[i], c = v[i + h];
-          v[i] = a + c;
-          v[i + h] = a - c;
+      for (int j = 0; j < NCH / 2; ++j) {
+        uint4 lo = make_uint4(0u, 0u, 0u, 0u), hi = make_uint4(0u, 0u, 0u, 0u);
+        if (valid) {
+          lo = *reinterpret_cast<const uint4*>(src + ((j ^ L) << 4));
+          hi = *reinterpret_cast<const uint4*>(src + (((j + NCH / 2) ^ L) << 4));
         }
+#pragma unroll
+        for (int e = 0; e < C; ++e) {
+          float a = elem(lo, e, x);
+          float b = elem(hi, e, x);
+          if (ACT == 1) {
+            a = gelu_erf(a);
+            b = gelu_erf(b);
+          }
+          V[j * C + e] = pk2(a, b);
+        }
+      }
+    }
+
+    // Walsh-Hadamard butterflies: distances 1..32 on the pairs, 64 inside a pair.
+    fht_stage2<1>(V);
+    fht_stage2<2>(V);
+    fht_stage2<4>(V);
+    fht_stage2<8>(V);
+    fht_stage2<16>(V);
+    fht_stage2<32>(V);
+    if (G >= 128) {
+#pragma unroll
+      for (int i = 0; i < kHalf; ++i) {
+        float a, b;
+        upk2(V[i], a, b);
+        V[i] = pk2(a + b, a - b);
       }
     }
     if (G == 256) {
       // Last stage across the two slabs of a group, held by lanes l and l^1
       // (their swizzles L differ in bit 0, so chunk j carries the relative
-      // sign (-1)^j).  Lower slab: a + b; upper slab: a - b.
-      const float self_sign = (s & 1) ? -1.0f : 1.0f;
+      // sign (-1)^j; both halves of V[i] lie in chunks of the same parity).
+      // Lower slab: a + b; upper slab: a - b.
+      const float ss = (s & 1) ? -1.0f : 1.0f;
+      const uint64_t ss2 = pk2(ss, ss);
 #pragma unroll
-      for (int j = 0; j < NCH; ++j) {
-#pragma unroll
-        for (int e = 0; e < C; ++e) {
-          const int i = j * C + e;
-          const float other = __shfl_xor_sync(0xFFFFFFFFu, v[i], 1);
-          const float t = (j & 1) ? -other : other;
-          v[i] = fmaf(v[i], self_sign, t);
-        }
+      for (int i = 0; i < kHalf; ++i) {
+        const uint64_t other = __shfl_xor_sync(0xFFFFFFFFu, V[i], 1);
+        V[i] = ((i / C) & 1) ? sub2(mul2(V[i], ss2), other) : fma2(V[i], ss2, other);
       }
     }
+    float am[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int i = 0; i < kSlab; ++i) amax = fmaxf(amax, fabsf(v[i]));
-    if (valid && ok) atomicMax(&row_amax[it & 1][p], __float_as_uint(amax * norm));
-    __syncthreads();
-    if (tid < 64) row_amax[(it + 1) & 1][tid] = 0u;   // next tile's slots (last read a tile ago)
+    for (int i = 0; i < kHalf; ++i) {
+      float a, b;
+      upk2(V[i], a, b);
+      am[i & 7] = fmaxf(am[i & 7], fmaxf(fabsf(a), fabsf(b)));
+    }
+    const float amax = fmaxf(fmaxf(fmaxf(am[0], am[1]), fmaxf(am[2], am[3])),
+                             fmaxf(fmaxf(am[4], am[5]), fmaxf(am[6], am[7])));
+    // max_k fl(|u_k| * norm) = fl(max_k |u_k| * norm): rounding is monotonic
+    if (valid) atomicMax(&row_amax[it % 3][p], __float_as_uint(amax * norm));
+    __syncthreads();   // every thread has its slab: ring slot st is free again
+    if (abort_flag) break;
+    if (tid == 0) {
+      const int64_t nt = tile + static_cast<int64_t>(nstages) * gridDim.x;
+      if (nt < ntiles) {
+        issue(nt, st);
+        ++issued;
+      }
+    }
+    // slots of it % 3 are read below; those of (it + 2) % 3 were last read in
+    // the previous tile and are next written after the coming barrier
+    if (tid < P) row_amax[(it + 2) % 3][tid] = 0u;
+    if (!valid) continue;
 
-    if (valid && ok) {
-      const float amax_r = __uint_as_float(row_amax[it & 1][p]);
-      const float sc = amax_r / 7.0f;                  // fp32 division, as the method states
-      if (s == 0) scale[row] = sc;
-      uint32_t packed[kSlab / 8];
-      if (sc > 0.0f) {
-        const float inv = 1.0f / sc;
+    const float amax_r = __uint_as_float(row_amax[it % 3][p]);
+    const float sc = amax_r / 7.0f;   // fp32 division, as the method states
+    if (s == 0) scale[row] = sc;
+    uint32_t packed[kSlab / 8];
+    if (sc > 0.0f) {
+      const float ni = norm * (1.0f / sc);
+      const uint64_t magic2 = pk2(kMagic8, kMagic8);
+      const uint64_t near2 = pk2(-kNearSq, -kNearSq);
+      uint32_t fb[kSlab];            // float bits of q + kMagic8, slot order
+      uint32_t signs = 0xFFFFFFFFu;  // AND of the near-test results
 #pragma unroll
-        for (int j = 0; j < NCH; ++j) {
-          // sign of output chunk j: (-1)^popcount(j & L)
-          const float sgn = (__popc(j & L) & 1) ? -1.0f : 1.0f;
-          const float mul = norm * inv * sgn;
+      for (int i = 0; i < kHalf; ++i) {
+        // sign of output chunk i / C (both halves share it, since L < 8)
+        const float m = (__popc((i / C) & L) & 1) ? -ni : ni;
+        const uint64_t q = mul2(V[i], pk2(m, m));
+        const uint64_t f = add2(q, magic2);
+        const uint64_t d = sub2(q, sub2(f, magic2));
+        const uint64_t t = fma2(d, d, near2);
+        float t0, t1, f0, f1;
+        upk2(t, t0, t1);
+        upk2(f, f0, f1);
+        signs &= __float_as_uint(t0) & __float_as_uint(t1);
+        fb[i] = __float_as_uint(f0);
+        fb[i + kHalf] = __float_as_uint(f1);
+      }
 #pragma unroll
-          for (int e = 0; e < C; ++e) {
-            const int i = j * C + e;
-            float q = v[i] * mul;
-            float k = rintf(q);
-            // Near a rounding boundary take the decision on r / s exactly.
-            if (fabsf(q - k) > 0.5f - 4e-7f * fabsf(q) - 1e-30f) {
-              const float r = __fmul_rn(v[i] * sgn, norm);
-              k = rintf(__fdiv_rn(r, sc));
-            }
-            v[i] = k;
+      for (int w = 0; w < kSlab / 8; ++w) {
+        uint32_t acc = fb[8 * w + 7];
+#pragma unroll
+        for (int e = 6; e >= 0; --e) acc = acc * 16u + fb[8 * w + e];
+        packed[w] = (acc - kHornerBias) ^ 0x88888888u;
+      }
+      // a near-test result >= 0 (sign bit clear) marks a code next to a
+      // rounding boundary: decide those codes again exactly
+      if ((signs & 0x80000000u) == 0u) {
+        float vl[kSlab];
+        uint32_t pl[kSlab / 8];
+#pragma unroll
+        for (int i = 0; i < kHalf; ++i) upk2(V[i], vl[i], vl[i + kHalf]);
+#pragma unroll
+        for (int w = 0; w < kSlab / 8; ++w) pl[w] = packed[w];
+#pragma unroll 1
+        for (int i = 0; i < kSlab; ++i) {
+          const bool neg = (__popc(((i & (kHalf - 1)) / C) & L) & 1) != 0;
+          const float q = vl[i] * (neg ? -ni : ni);
+          const float f = q + kMagic8;
+          const float dd = q - (f - kMagic8);
+          if (__fmaf_rn(dd, dd, -kNearSq) >= 0.0f) {
+            const uint32_t nib = exact_code(neg ? -vl[i] : vl[i], norm, sc, q);
+            const int sh = 4 * (i & 7);
+            pl[i >> 3] = (pl[i >> 3] & ~(0xFu << sh)) | (nib << sh);
           }
         }
 #pragma unroll
-        for (int w = 0; w < kSlab / 8; ++w) {
-          uint32_t word = 0;
-#pragma unroll
-          for (int e = 0; e < 8; ++e) word |= (static_cast<uint32_t>(static_cast<int>(v[w * 8 + e])) & 0xFu) << (4 * e);
-          packed[w] = word;
-        }
-      } else {
-#pragma unroll
-        for (int w = 0; w < kSlab / 8; ++w) packed[w] = 0u;
+        for (int w = 0; w < kSlab / 8; ++w) packed[w] = pl[w];
       }
-      uint4* dst = reinterpret_cast<uint4*>(out + row * static_cast<int64_t>(K / 2) + static_cast<int64_t>(s) * (kSlab / 2));
+    } else {
 #pragma unroll
-      for (int w = 0; w < kSlab / 32; ++w)
-        dst[w] = make_uint4(packed[4 * w], packed[4 * w + 1], packed[4 * w + 2], packed[4 * w + 3]);
+      for (int w = 0; w < kSlab / 8; ++w) packed[w] = 0u;
     }
-    __syncthreads();   // buffer b and row_amax[it & 1] are free after this
-    if (abort_flag) break;
+    uint4* dst = reinterpret_cast<uint4*>(out + row * static_cast<int64_t>(K / 2) +
+                                          static_cast<int64_t>(s) * (kSlab / 2));
+#pragma unroll
+    for (int w = 0; w < kSlab / 32; ++w)
+      dst[w] = make_uint4(packed[4 * w], packed[4 * w + 1], packed[4 * w + 2], packed[4 * w + 3]);
   }
-  // After an abort, let any copy this CTA issued land before it exits.
-  if (abort_flag && tid == 0) {
-    (void)mbar_wait(&full_bar[0], 0, nullptr, nullptr, 1000000ull);
-    (void)mbar_wait(&full_bar[1], 0, nullptr, nullptr, 1000000ull);
+  // After an abort, let every copy thread 0 issued land before the CTA exits.
+  if (tid == 0 && abort_flag) {
+    for (int st = 0; st < nstages && st < issued; ++st) {
+      const int64_t n_st = issued / nstages + (st < issued % nstages ? 1 : 0);
+      (void)mbar_wait(&full[st], static_cast<uint32_t>((n_st - 1) & 1), nullptr, nullptr, 100000000ull);
+    }
   }
 }
 
-// Host-side launch.  Returns a cudaError_t.
+// Rows per tile and threads per CTA for a row of S slabs: as many whole rows
+// as fit in the thread limit (at most kMaxRows).
+static void rq_shape(int S, int max_threads, int* P, int* threads) {
+  int p = max_threads / S;
+  if (p < 1) p = 1;
+  if (p > kMaxRows) p = kMaxRows;
+  *P = p;
+  *threads = ((p * S + 31) / 32) * 32;
+}
+
 template <typename TIn, int G, int ACT>
-static cudaError_t launch_rq(const TIn* x, int64_t M, int K, int64_t ldx, int8_t* out, float* scale,
-                             int num_sms, unsigned int* status, cudaStream_t stream) {
+static cudaError_t launch_rq(const TIn* x, int64_t M, int K, int64_t ldx, int8_t* out, float* scale, int num_sms,
+                             unsigned int* status, cudaStream_t stream) {
   const int S = K / kSlab;
-  const int maxT = InTraits<TIn>::kMaxThreads;
-  int P = maxT / S;
-  if (P < 1) return cudaErrorInvalidValue;
-  if (P > 64) P = 64;
-  if (G == 256 && (P * S) % 2) --P;  // never happens (S is even for g = 256)
-  int threads = ((P * S + 31) / 32) * 32;
-  const size_t smem = 2 * static_cast<size_t>(P) * K * sizeof(TIn);
+  if (S > InTraits<TIn>::kMaxThreads) return cudaErrorInvalidValue;
+  int P, threads;
+  rq_shape(S, InTraits<TIn>::kMaxThreads, &P, &threads);
+  const size_t stage_bytes = static_cast<size_t>(P) * K * sizeof(TIn);
+  int nst = static_cast<int>(kRingBytes / stage_bytes);
+  if (nst > kMaxStages) nst = kMaxStages;
+  if (nst < 1) return cudaErrorInvalidValue;
+  const size_t smem = nst * stage_bytes;
   auto kern = rotate_quant_pack_kernel<TIn, G, ACT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  const int64_t ntiles = (M + P - 1) / P;
-  const int grid = static_cast<int>(ntiles < num_sms ? ntiles : num_sms);
-  kern<<<grid, threads, smem, stream>>>(x, M, K, ldx, P, out, scale, status);
+  const int64_t tiles = (M + P - 1) / P;
+  const int64_t grid = tiles < num_sms ? tiles : num_sms;
+  kern<<<static_cast<unsigned>(grid), threads, smem, stream>>>(x, M, K, ldx, P, nst, out, scale, status);
   return cudaGetLastError();
 }
 

@@ -65,29 +65,29 @@ struct Bars {
   unsigned int last;
 };
 
-__device__ __forceinline__ void widen_word(uint32_t w, uint32_t& o0, uint32_t& o1) {
-  uint32_t lo = w & 0x0F0F0F0Fu;
-  uint32_t hi = (w >> 4) & 0x0F0F0F0Fu;
-  lo = (lo + 0x78787878u) ^ 0x78787878u;
-  hi = (hi + 0x78787878u) ^ 0x78787878u;
-  o0 = __byte_perm(lo, hi, 0x5140);
-  o1 = __byte_perm(lo, hi, 0x7362);
+// Same widening as the large-M kernel: each nibble q lands in the high half of
+// a byte (the signed byte 16*q); both operands share the byte order, the MMA
+// accumulates 256*acc exactly and the epilogue shifts the factor out.
+__device__ __forceinline__ void widen_word16(uint32_t w, uint32_t& o0, uint32_t& o1) {
+  o0 = w & 0xF0F0F0F0u;
+  o1 = (w << 4) & 0xF0F0F0F0u;
 }
 
 template <int kUnits>
 __device__ __forceinline__ void widen_tile(const uint8_t* __restrict__ packed, uint8_t* __restrict__ wide, int wt) {
+  constexpr int kPer = (kUnits + kWorkWarps * 32 - 1) / (kWorkWarps * 32);
 #pragma unroll
-  for (int i = 0; i < (kUnits + kWorkWarps * 32 - 1) / (kWorkWarps * 32); ++i) {
+  for (int i = 0; i < kPer; ++i) {
     const int u = wt + i * kWorkWarps * 32;
     if (kUnits % (kWorkWarps * 32) != 0 && u >= kUnits) break;
     const int r = u >> 2;
     const int part = u & 3;
     const uint4 w = *reinterpret_cast<const uint4*>(packed + u * 16);
     uint4 c0, c1;
-    widen_word(w.x, c0.x, c0.y);
-    widen_word(w.y, c0.z, c0.w);
-    widen_word(w.z, c1.x, c1.y);
-    widen_word(w.w, c1.z, c1.w);
+    widen_word16(w.x, c0.x, c0.y);
+    widen_word16(w.y, c0.z, c0.w);
+    widen_word16(w.z, c1.x, c1.y);
+    widen_word16(w.w, c1.z, c1.w);
     uint8_t* rowp = wide + (r >> 3) * 1024 + (r & 7) * 128;
     const int sw = r & 7;
     *reinterpret_cast<uint4*>(rowp + (((2 * part) ^ sw) << 4)) = c0;
@@ -210,9 +210,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t ps = 0, ph = 0, ws = 0, wph = 0;
     bool ok = true;
     for (int i = 0; i < nkb; ++i) {
-      bool got = mbar_wait(&bars.packed_full[ps], ph, abort_flag, args.status);
-      got = got && mbar_wait(&bars.wide_empty[ws], wph ^ 1, abort_flag, args.status);
-      if (!__all_sync(0xFFFFFFFFu, got)) { ok = false; break; }
+      if (!warp_wait(&bars.packed_full[ps], ph, abort_flag, args.status) ||
+          !warp_wait(&bars.wide_empty[ws], wph ^ 1, abort_flag, args.status)) { ok = false; break; }
       widen_tile<WM * BKP / 16>(smem + Lay::kOffPackW + ps * Lay::kPackW, smem + Lay::kOffWideW + ws * Lay::kWideW, wt);
       widen_tile<NP * BKP / 16>(smem + Lay::kOffPackX + ps * Lay::kPackX, smem + Lay::kOffWideX + ws * Lay::kWideX, wt);
       fence_async_shared();
@@ -225,7 +224,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (++ws == SWD) { ws = 0; wph ^= 1; }
     }
     // ------------------------------------------------------------- epilogue
-    if (ok) (void)mbar_wait(&bars.acc_full, 0, abort_flag, args.status);
+    if (ok) (void)warp_wait(&bars.acc_full, 0, abort_flag, args.status);
     // the four work warps agree before any of them takes the named barriers below
     asm volatile("bar.sync 1, %0;" ::"r"(kWorkWarps * 32) : "memory");
     const bool all_ok = *abort_flag == 0;
@@ -238,6 +237,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       tmem_ld_cols<NP>(tmem_base + (static_cast<uint32_t>(q * 32) << 16), acc);
       tmem_wait_ld();
+#pragma unroll
+      for (int m = 0; m < NP; ++m) acc[m] = static_cast<uint32_t>(static_cast<int32_t>(acc[m]) >> 8);
     }
     const int mrows = static_cast<int>(M);
     bool do_epi = all_ok && splits == 1;

@@ -14,9 +14,10 @@ cudaError_t rotate_quant_bf16(const uint16_t* x, int64_t M, int K, int64_t ldx, 
                               float* scale, int num_sms, unsigned int* status, cudaStream_t stream);
 cudaError_t rotate_quant_f32(const float* x, int64_t M, int K, int64_t ldx, int g, int8_t* out, float* scale,
                              int num_sms, unsigned int* status, cudaStream_t stream);
-// Largest K the in-register rotate kernel supports: 384 threads x 128 codes
-// for bf16 rows, 192 threads x 128 codes for fp32 rows (weights).
-constexpr int kQuantMaxK = 384 * 128;
+// Largest K the in-register rotate kernel supports (one row per CTA at most):
+// 256 threads x 128 codes for bf16 rows, 192 threads x 128 codes for fp32
+// rows (weights).
+constexpr int kQuantMaxK = 256 * 128;
 constexpr int kQuantMaxKF32 = 192 * 128;
 
 // ---- tcgen05 GEMM (gemm.cu)
@@ -30,11 +31,11 @@ struct GemmArgs {
   int out_s32;            // 1: raw int32 accumulators
   unsigned int* status;   // device status word (bounded-wait timeouts)
 };
-// tmA: packed activations [M, K/2] bytes, box {64, 128}; tmB: packed weights
-// [N, K/2] bytes, box {64, 256}.
-cudaError_t gemm_tc_launch(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a, int num_sms,
+// xq: packed activations [M, K/2] bytes; wq: packed weights [N, K/2] bytes
+// (contiguous rows, 16-byte aligned).  Launched as clusters of 2 CTAs.
+cudaError_t gemm_tc_launch(const int8_t* xq, const int8_t* wq, const GemmArgs& a, int num_sms,
                            cudaStream_t stream);
-constexpr int kGemmBM = 128;
+constexpr int kGemmBM = 256;
 constexpr int kGemmBN = 256;
 
 // ---- small-M weight-streaming GEMM (smallm.cu)
