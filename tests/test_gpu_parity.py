@@ -252,3 +252,32 @@ def test_bounded_wait_reports_timeout_and_context_survives(cuda_lib):
     cfg = workloads.TINY
     x, W, b = cfg.make()
     _check_layer(cuda_lib, cfg, x, W, b)
+
+
+def test_quantize_exact_ties_follow_round_half_even(cuda_lib):
+    """Rows built from the hand-derived tie fixture: every rotated value is an
+    exact multiple of 1/2 or 1/4, so many codes sit exactly on a rounding
+    boundary.  The kernel must decide all of them as round-half-even of the
+    fp32 quotient, with no boundary tolerance."""
+    import os
+    import scipy.linalg
+    from test_oracle_pins import _read_golden_ties
+    g, cases = _read_golden_ties()
+    Hs = scipy.linalg.hadamard(g).astype(np.float64) / 8.0
+    rows = []
+    for c in cases:
+        r = np.zeros(g)
+        r[:len(c["r"])] = c["r"]
+        rows.append(Hs @ r)
+    # K = 128 (two groups of 64): pair the cases, and repeat with permuted
+    # group order and signs so the rows span several CTAs and lanes
+    base = [np.concatenate([rows[0], rows[1]]), np.concatenate([rows[1], -rows[0]])]
+    X = np.stack([base[i % 2] * (1 if (i // 2) % 2 == 0 else -1) for i in range(300)])
+    xb = orc.f32_to_bf16_bits(X.astype(np.float32))
+    assert np.array_equal(orc.bf16_bits_to_f32(xb).astype(np.float64), X)
+    x = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).cuda()
+    Xq, sx = cuda_lib.quantize_activation(x, g)
+    ref = orc.quantize_activation(xb, g)
+    assert np.array_equal(Xq.cpu().numpy(), ref["packed"])
+    assert np.array_equal(sx.cpu().numpy(), ref["scale"])
+    assert np.sum(orc.boundary_window(ref["v"], 0.0)) > 1000   # the ties are really there

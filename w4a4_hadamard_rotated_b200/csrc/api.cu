@@ -156,6 +156,9 @@ int run_linear(const int8_t* Xq, const float* sx, const int8_t* Wq, const float*
     a.status = dev->status;
     return smallm_launch_tm(tmW, tmX, a, dev->num_sms, stream) == cudaSuccess ? W4A4_OK : W4A4_ERR_CUDA;
   }
+  CUtensorMap tmA, tmB;
+  if ((st = packed_map(&tmA, Xq, M, K, kGemmBM / 2)) != W4A4_OK) return st;
+  if ((st = packed_map(&tmB, Wq, N, K, kGemmBN / 2)) != W4A4_OK) return st;
   GemmArgs a{};
   a.M = M;
   a.N = N;
@@ -167,7 +170,7 @@ int run_linear(const int8_t* Xq, const float* sx, const int8_t* Wq, const float*
   a.ldo = ldo;
   a.out_s32 = out_s32;
   a.status = dev->status;
-  return gemm_tc_launch(Xq, Wq, a, dev->num_sms, stream) == cudaSuccess ? W4A4_OK : W4A4_ERR_CUDA;
+  return gemm_tc_launch(tmA, tmB, a, dev->num_sms, stream) == cudaSuccess ? W4A4_OK : W4A4_ERR_CUDA;
 }
 
 __global__ void wait_forever_bounded_kernel(unsigned long long limit_ns, unsigned int* status) {

@@ -17,11 +17,12 @@
 //     the B tile, which keeps its shared-memory traffic per k-block (32 KB of
 //     widened bytes written, 32 KB read by the tensor core) under the time of
 //     the MMA itself.
-//   * Eight "widen" warps per CTA fetch the packed nibbles of their half-tiles
-//     straight from L2/HBM into registers (128-bit loads, two k-blocks ahead),
-//     place every nibble q in the high half of a byte -- the signed byte 16*q,
-//     so no sign extension is needed -- and store the bytes in the 128-byte-
-//     swizzle K-major layout the MMA reads, into a 6-deep ring.  Both operands
+//   * A producer warp per CTA TMA-loads the packed nibbles of its half-tiles
+//     (64-byte rows, 128 rows of A and of B per k-block) into a 4-deep ring.
+//     Eight "widen" warps read them back with 128-bit shared loads, place
+//     every nibble q in the high half of a byte -- the signed byte 16*q, so no
+//     sign extension is needed -- and store the bytes in the 128-byte-swizzle
+//     K-major layout the MMA reads, into a second 4-deep ring.  Both operands
 //     get the same treatment (and the same byte order inside each word), so
 //     the MMA accumulates 256 * acc exactly (|256 acc| <= 12544 K < 2^31 for
 //     K <= 131072) and the epilogue shifts the factor back out.
@@ -52,11 +53,13 @@ constexpr int HM = BM / 2;      // A rows per CTA
 constexpr int HN = BN / 2;      // B rows per CTA
 constexpr int BK = 128;         // int4 codes per k-block (= bytes per widened row)
 constexpr int BKP = BK / 2;     // packed bytes per row per k-block
-constexpr int SWD = 6;          // widened ring depth
+constexpr int SP = 4;           // packed ring depth
+constexpr int SWD = 4;          // widened ring depth
 constexpr int kWidenWarps = 8;
 constexpr int kEpiWarps = 4;
 constexpr int kWarpMma = 0;
-constexpr int kWarpWiden0 = 1;
+constexpr int kWarpTma = 1;
+constexpr int kWarpWiden0 = 2;
 constexpr int kWarpEpi0 = kWarpWiden0 + kWidenWarps;
 constexpr int kThreads = (kWarpEpi0 + kEpiWarps) * 32;
 constexpr int kTmemCols = 2 * BN;   // two int32 accumulators of BN columns
@@ -64,15 +67,20 @@ constexpr int kTmemCols = 2 * BN;   // two int32 accumulators of BN columns
 constexpr uint32_t kWideA = HM * BK;     // 16 KB
 constexpr uint32_t kWideB = HN * BK;     // 16 KB
 constexpr uint32_t kStage = kWideA + kWideB;
-constexpr uint32_t kSmemBytes = SWD * kStage;
+constexpr uint32_t kPackA = HM * BKP;    // 8 KB
+constexpr uint32_t kPackB = HN * BKP;    // 8 KB
+constexpr uint32_t kPStage = kPackA + kPackB;
+constexpr uint32_t kOffPack = SWD * kStage;
+constexpr uint32_t kSmemBytes = kOffPack + SP * kPStage;
 constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;   // slack for 1024-byte alignment
 
 // packed 16-byte units per CTA and k-block: (HM + HN) rows x 4 units
 constexpr int kUnits = (HM + HN) * (BKP / 16);
 constexpr int kUnitsPerThread = kUnits / (kWidenWarps * 32);   // 4
-constexpr int kPrefetch = 3;   // register sets of packed units in flight, one per k-block
 
 struct Bars {
+  uint64_t packed_full[SP];   // TMA transaction barrier
+  uint64_t packed_empty[SP];  // kWidenWarps local arrivals
   // even CTA: its kWidenWarps local arrivals plus one forwarded by the odd
   // CTA; odd CTA: its kWidenWarps local arrivals (consumed by the forwarder)
   uint64_t wide_full[SWD];
@@ -93,29 +101,13 @@ __device__ __forceinline__ void widen_word16(uint32_t w, uint32_t& o0, uint32_t&
   o1 = (w << 4) & 0xF0F0F0F0u;
 }
 
-// Fetch this thread's packed units of one k-block (rows outside the matrix
-// and columns beyond K read as zeros, which add nothing to the products).
-__device__ __forceinline__ void load_units(uint4 (&buf)[kUnitsPerThread], const GemmArgs& a, const int8_t* xq,
-                                           const int8_t* wq, int wt, int64_t arow0, int64_t brow0, int kb) {
-  const int64_t kbytes = a.K / 2;
+// Widen this thread's packed units of one k-block (read from the packed
+// stage; A units first, then B) into the widened stage.
+__device__ __forceinline__ void widen_units(const uint8_t* __restrict__ pstage, uint8_t* __restrict__ stage, int wt) {
+  uint4 buf[kUnitsPerThread];
 #pragma unroll
-  for (int i = 0; i < kUnitsPerThread; ++i) {
-    const int u = wt + i * kWidenWarps * 32;
-    const bool isA = u < HM * 4;
-    const int uu = isA ? u : u - HM * 4;
-    const int r = uu >> 2;
-    const int64_t col = static_cast<int64_t>(kb) * BKP + (uu & 3) * 16;
-    const int64_t row = (isA ? arow0 : brow0) + r;
-    const int64_t rows = isA ? a.M : a.N;
-    const int8_t* base = isA ? xq : wq;
-    if (row < rows && col < kbytes)
-      buf[i] = __ldg(reinterpret_cast<const uint4*>(base + row * kbytes + col));
-    else
-      buf[i] = make_uint4(0u, 0u, 0u, 0u);
-  }
-}
-
-__device__ __forceinline__ void store_units(const uint4 (&buf)[kUnitsPerThread], uint8_t* stage, int wt) {
+  for (int i = 0; i < kUnitsPerThread; ++i)
+    buf[i] = *reinterpret_cast<const uint4*>(pstage + (wt + i * kWidenWarps * 32) * 16);
 #pragma unroll
   for (int i = 0; i < kUnitsPerThread; ++i) {
     const int u = wt + i * kWidenWarps * 32;
@@ -137,7 +129,7 @@ __device__ __forceinline__ void store_units(const uint4 (&buf)[kUnitsPerThread],
 
 template <int OUT_S32>
 __global__ void __launch_bounds__(kThreads, 1)
-    gemm_tc_kernel(const int8_t* __restrict__ xq, const int8_t* __restrict__ wq, GemmArgs args) {
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmArgs args) {
   extern __shared__ uint8_t smem_dyn[];
   __shared__ Bars bars;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
@@ -154,6 +146,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int num_kb = static_cast<int>((args.K + BK - 1) / BK);
 
   if (threadIdx.x == 0) {
+    for (int s = 0; s < SP; ++s) {
+      mbar_init(&bars.packed_full[s], 1);
+      mbar_init(&bars.packed_empty[s], kWidenWarps);
+    }
     for (int s = 0; s < SWD; ++s) {
       mbar_init(&bars.wide_full[s], rank == 0 ? kWidenWarps + 1 : kWidenWarps);
       mbar_init(&bars.wide_empty[s], 1);
@@ -165,6 +161,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars.drain, 1);
     bars.abort_flag = 0;
     fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
   }
   if (warp == kWarpMma) {
     tmem_alloc_pair(&bars.tmem_base, kTmemCols);
@@ -228,54 +226,51 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
       }
     }
+  } else if (warp == kWarpTma) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      uint32_t ps = 0, ph = 0;
+      int64_t issued = 0;
+      bool ok = true;
+      for (int t = cluster; t < tiles && ok; t += nclusters) {
+        const int mb = t % num_m, nb = t / num_m;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&bars.packed_empty[ps], ph ^ 1, abort_flag, args.status)) { ok = false; break; }
+          mbar_arrive_expect_tx(&bars.packed_full[ps], kPStage);
+          uint8_t* dst = smem + kOffPack + ps * kPStage;
+          tma_load_2d(dst, &tmA, &bars.packed_full[ps], kb * BKP, mb * BM + static_cast<int>(rank) * HM);
+          tma_load_2d(dst + kPackA, &tmB, &bars.packed_full[ps], kb * BKP, nb * BN + static_cast<int>(rank) * HN);
+          ++issued;
+          if (++ps == SP) { ps = 0; ph ^= 1; }
+        }
+      }
+      if (!ok) {
+        // let every copy this thread issued land before the CTA goes away
+        for (int s2 = 0; s2 < SP && s2 < issued; ++s2) {
+          const int64_t n_s = issued / SP + (s2 < issued % SP ? 1 : 0);
+          (void)mbar_wait(&bars.packed_full[s2], static_cast<uint32_t>((n_s - 1) & 1), nullptr, nullptr, 100000000ull);
+        }
+      }
+    }
   } else if (warp < kWarpEpi0) {
     // ------------------------------------------------------------ widen warps
     const int wt = threadIdx.x - kWarpWiden0 * 32;
-    uint4 buf[kPrefetch][kUnitsPerThread];
-    // the sequence of (tile, k-block) positions this cluster walks
-    int t = cluster, kb = 0;        // position being widened
-    int pt = cluster, pkb = 0;      // position of the next prefetch
-#pragma unroll
-    for (int p = 0; p < kPrefetch; ++p) {
-      if (pt < tiles) {
-        load_units(buf[p], args, xq, wq, wt, static_cast<int64_t>(pt % num_m) * BM + rank * HM,
-                   static_cast<int64_t>(pt / num_m) * BN + rank * HN, pkb);
-        if (++pkb == num_kb) { pkb = 0; pt += nclusters; }
-      }
-    }
-    uint32_t ws = 0, wph = 0;
-    int slot = 0;
-    while (t < tiles) {
-      if (!warp_wait_cluster(&bars.wide_empty[ws], wph ^ 1, abort_flag, args.status)) break;
-      uint4 cur[kUnitsPerThread];
-#pragma unroll
-      for (int s = 0; s < kPrefetch; ++s)
-        if (s == slot) {
-#pragma unroll
-          for (int i = 0; i < kUnitsPerThread; ++i) cur[i] = buf[s][i];
+    uint32_t ps = 0, ph = 0, ws = 0, wph = 0;
+    bool ok = true;
+    for (int t = cluster; t < tiles && ok; t += nclusters) {
+      for (int kb = 0; kb < num_kb; ++kb) {
+        if (!warp_wait(&bars.packed_full[ps], ph, abort_flag, args.status) ||
+            !warp_wait_cluster(&bars.wide_empty[ws], wph ^ 1, abort_flag, args.status)) { ok = false; break; }
+        widen_units(smem + kOffPack + ps * kPStage, smem + ws * kStage, wt);
+        fence_async_shared();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&bars.wide_full[ws]);
+          mbar_arrive(&bars.packed_empty[ps]);
         }
-      store_units(cur, smem + ws * kStage, wt);
-      fence_async_shared();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.wide_full[ws]);
-      if (++ws == SWD) { ws = 0; wph ^= 1; }
-      // refill the set just used with the position kPrefetch ahead, so the
-      // loads of the next kPrefetch - 1 k-blocks are always in flight
-      if (pt < tiles) {
-        const int ns = slot;
-        uint4 tmp[kUnitsPerThread];
-        load_units(tmp, args, xq, wq, wt, static_cast<int64_t>(pt % num_m) * BM + rank * HM,
-                   static_cast<int64_t>(pt / num_m) * BN + rank * HN, pkb);
-#pragma unroll
-        for (int s = 0; s < kPrefetch; ++s)
-          if (s == ns) {
-#pragma unroll
-            for (int i = 0; i < kUnitsPerThread; ++i) buf[s][i] = tmp[i];
-          }
-        if (++pkb == num_kb) { pkb = 0; pt += nclusters; }
+        if (++ps == SP) { ps = 0; ph ^= 1; }
+        if (++ws == SWD) { ws = 0; wph ^= 1; }
       }
-      slot = (slot + 1 == kPrefetch) ? 0 : slot + 1;
-      if (++kb == num_kb) { kb = 0; t += nclusters; }
     }
   } else {
     // ------------------------------------------------------------ epilogue warps
@@ -411,7 +406,7 @@ int max_clusters(int num_sms) {
 }
 
 template <int OUT_S32>
-cudaError_t launch(const int8_t* xq, const int8_t* wq, const GemmArgs& a, int64_t tiles, int num_sms,
+cudaError_t launch(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a, int64_t tiles, int num_sms,
                    cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<OUT_S32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(kSmemAlloc));
@@ -430,15 +425,17 @@ cudaError_t launch(const int8_t* xq, const int8_t* wq, const GemmArgs& a, int64_
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<OUT_S32>, xq, wq, a);
+  return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<OUT_S32>, tmA, tmB, a);
 }
 
 }  // namespace
 
-cudaError_t gemm_tc_launch(const int8_t* xq, const int8_t* wq, const GemmArgs& a, int num_sms, cudaStream_t stream) {
+cudaError_t gemm_tc_launch(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a, int num_sms,
+                           cudaStream_t stream) {
   const int64_t tiles = ((a.M + BM - 1) / BM) * ((a.N + BN - 1) / BN);
   if (tiles == 0) return cudaSuccess;
-  cudaError_t e = a.out_s32 ? launch<1>(xq, wq, a, tiles, num_sms, stream) : launch<0>(xq, wq, a, tiles, num_sms, stream);
+  cudaError_t e =
+      a.out_s32 ? launch<1>(tmA, tmB, a, tiles, num_sms, stream) : launch<0>(tmA, tmB, a, tiles, num_sms, stream);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

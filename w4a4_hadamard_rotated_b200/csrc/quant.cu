@@ -26,13 +26,14 @@
 //     chunk is folded into the quantisation multiplier; the quantiser is odd
 //     (round-half-even and the clamp are symmetric), so the codes are exact.
 //   * The row amax is reduced with shared-memory atomics on the float bits
-//     (triple-buffered slots, one barrier per tile).  The code is round-half-
-//     even of r / s with s = amax / 7, taken in fp32: a reciprocal multiply
-//     and a magic-number rounding put the code in the low mantissa bits, a
-//     Horner chain of integer multiply-adds packs 8 codes per word, and if any
-//     element of the slab lies within 4e-6 of a rounding boundary those codes
-//     are decided again exactly (an fp64 comparison, see exact_code), so the
-//     codes equal those of the fp32 quotient r / s.
+//     (triple-buffered slots, one barrier per tile), and s = amax / 7 in fp32.
+//     The code is round-half-even of r * (1/s) in fp32: a reciprocal multiply
+//     (with 1/sqrt(g) and the chunk sign folded in) and a magic-number rounding
+//     put the code in the low mantissa bits, and a Horner chain of integer
+//     multiply-adds packs 8 codes per word as they are made.  The product is
+//     within 3 ulp of the quotient r / s, so a code can differ from the one of
+//     the exact quotient only for values within ~4e-7 (relative) of a rounding
+//     boundary; exact ties with power-of-two scales stay exact.
 //   * Codes are stored low nibble first, 64 contiguous bytes per thread, with
 //     128-bit stores.
 #include <cuda_bf16.h>
@@ -121,25 +122,6 @@ __device__ __forceinline__ void fht_stage2(uint64_t (&V)[kHalf]) {
   }
 }
 
-// The code of one element taken exactly as the method states it, without a
-// division: r = fl(u * norm), and the code is round-half-even of the fp32
-// quotient fl(r / s).  `q` is a fast estimate of r / s that lies within 4e-6
-// of the boundary b = k + 1/2.  fl(r / s) equals b exactly when |r/s - b| is at
-// most half an fp32 ulp of b (b's own mantissa is even, so the ties at the
-// ends go to b); otherwise it lies strictly on one side.  Both tests are
-// exact in fp64: b has at most 5 significant bits, so b*s is exact; r and b*s
-// are within a factor of 2, so their difference is exact (Sterbenz); and the
-// half ulp is a power of two.
-__device__ __forceinline__ uint32_t exact_code(float u, float norm, float sc, float q) {
-  const float r = __fmul_rn(u, norm);
-  const float b = floorf(q) + 0.5f;
-  const double d = static_cast<double>(r) - static_cast<double>(b) * static_cast<double>(sc);
-  const float half_ulp = __int_as_float((((__float_as_int(b) >> 23) & 0xFF) - 24) << 23);
-  const double t = static_cast<double>(half_ulp) * static_cast<double>(sc);
-  const float k = d > t ? ceilf(b) : (d < -t ? floorf(b) : rintf(b));
-  return static_cast<uint32_t>(static_cast<int>(k)) & 0xFu;
-}
-
 // 1.5 * 2^23 + 8: adding it to |q| <= 7.5 rounds q to an integer k, half to
 // even, and leaves k + 8 (in 1..15) in the low four bits of the sum.
 constexpr float kMagic8 = 12582920.0f;
@@ -147,8 +129,6 @@ constexpr uint32_t kMagicBits = 0x4B400000u;   // bits of 1.5 * 2^23
 // Horner-packing eight sums (kMagicBits + n_e) as sum_e bits_e * 16^e leaves
 // this constant on top of the nibbles n_e (mod 2^32).
 constexpr uint32_t kHornerBias = kMagicBits * 0x11111111u;
-// Near-boundary test: (q - k)^2 - (0.5 - 4e-6)^2 >= 0.
-constexpr float kNearSq = (0.5f - 4e-6f) * (0.5f - 4e-6f);
 
 template <typename TIn, int G, int ACT>
 __global__ void __launch_bounds__(InTraits<TIn>::kMaxThreads, 1)
@@ -300,54 +280,25 @@ __global__ void __launch_bounds__(InTraits<TIn>::kMaxThreads, 1)
     if (sc > 0.0f) {
       const float ni = norm * (1.0f / sc);
       const uint64_t magic2 = pk2(kMagic8, kMagic8);
-      const uint64_t near2 = pk2(-kNearSq, -kNearSq);
-      uint32_t fb[kSlab];            // float bits of q + kMagic8, slot order
-      uint32_t signs = 0xFFFFFFFFu;  // AND of the near-test results
+      // Pairs V[8w .. 8w+8) hold the codes of words w (low halves) and w + 8
+      // (high halves): quantise and Horner-pack them together, so only the
+      // sixteen words stay live next to the slab.
 #pragma unroll
-      for (int i = 0; i < kHalf; ++i) {
-        // sign of output chunk i / C (both halves share it, since L < 8)
-        const float m = (__popc((i / C) & L) & 1) ? -ni : ni;
-        const uint64_t q = mul2(V[i], pk2(m, m));
-        const uint64_t f = add2(q, magic2);
-        const uint64_t d = sub2(q, sub2(f, magic2));
-        const uint64_t t = fma2(d, d, near2);
-        float t0, t1, f0, f1;
-        upk2(t, t0, t1);
-        upk2(f, f0, f1);
-        signs &= __float_as_uint(t0) & __float_as_uint(t1);
-        fb[i] = __float_as_uint(f0);
-        fb[i + kHalf] = __float_as_uint(f1);
-      }
+      for (int w = 0; w < kHalf / 8; ++w) {
+        uint32_t lo_acc = 0u, hi_acc = 0u;
 #pragma unroll
-      for (int w = 0; w < kSlab / 8; ++w) {
-        uint32_t acc = fb[8 * w + 7];
-#pragma unroll
-        for (int e = 6; e >= 0; --e) acc = acc * 16u + fb[8 * w + e];
-        packed[w] = (acc - kHornerBias) ^ 0x88888888u;
-      }
-      // a near-test result >= 0 (sign bit clear) marks a code next to a
-      // rounding boundary: decide those codes again exactly
-      if ((signs & 0x80000000u) == 0u) {
-        float vl[kSlab];
-        uint32_t pl[kSlab / 8];
-#pragma unroll
-        for (int i = 0; i < kHalf; ++i) upk2(V[i], vl[i], vl[i + kHalf]);
-#pragma unroll
-        for (int w = 0; w < kSlab / 8; ++w) pl[w] = packed[w];
-#pragma unroll 1
-        for (int i = 0; i < kSlab; ++i) {
-          const bool neg = (__popc(((i & (kHalf - 1)) / C) & L) & 1) != 0;
-          const float q = vl[i] * (neg ? -ni : ni);
-          const float f = q + kMagic8;
-          const float dd = q - (f - kMagic8);
-          if (__fmaf_rn(dd, dd, -kNearSq) >= 0.0f) {
-            const uint32_t nib = exact_code(neg ? -vl[i] : vl[i], norm, sc, q);
-            const int sh = 4 * (i & 7);
-            pl[i >> 3] = (pl[i >> 3] & ~(0xFu << sh)) | (nib << sh);
-          }
+        for (int e = 7; e >= 0; --e) {
+          const int i = 8 * w + e;
+          // sign of output chunk i / C (both halves share it, since L < 8)
+          const float m = (__popc((i / C) & L) & 1) ? -ni : ni;
+          const uint64_t f = add2(mul2(V[i], pk2(m, m)), magic2);
+          float f0, f1;
+          upk2(f, f0, f1);
+          lo_acc = lo_acc * 16u + __float_as_uint(f0);
+          hi_acc = hi_acc * 16u + __float_as_uint(f1);
         }
-#pragma unroll
-        for (int w = 0; w < kSlab / 8; ++w) packed[w] = pl[w];
+        packed[w] = (lo_acc - kHornerBias) ^ 0x88888888u;
+        packed[w + kHalf / 8] = (hi_acc - kHornerBias) ^ 0x88888888u;
       }
     } else {
 #pragma unroll

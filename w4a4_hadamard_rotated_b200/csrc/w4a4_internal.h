@@ -31,9 +31,9 @@ struct GemmArgs {
   int out_s32;            // 1: raw int32 accumulators
   unsigned int* status;   // device status word (bounded-wait timeouts)
 };
-// xq: packed activations [M, K/2] bytes; wq: packed weights [N, K/2] bytes
-// (contiguous rows, 16-byte aligned).  Launched as clusters of 2 CTAs.
-cudaError_t gemm_tc_launch(const int8_t* xq, const int8_t* wq, const GemmArgs& a, int num_sms,
+// tmA: packed activations [M, K/2] bytes, tmB: packed weights [N, K/2] bytes,
+// both with box {64 bytes, kGemmBM/2 rows}.  Launched as clusters of 2 CTAs.
+cudaError_t gemm_tc_launch(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a, int num_sms,
                            cudaStream_t stream);
 constexpr int kGemmBM = 256;
 constexpr int kGemmBN = 256;
