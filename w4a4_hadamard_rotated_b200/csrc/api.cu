@@ -91,6 +91,21 @@ int packed_map(CUtensorMap* map, const int8_t* base, int64_t rows, int64_t K, in
   return r == CUDA_SUCCESS ? W4A4_OK : W4A4_ERR_CUDA;
 }
 
+// 2-D map over a bf16 output [rows, cols] with row stride ld (elements), box
+// {32, 32}, 64-byte swizzle (the epilogue's staging layout).
+int output_map(CUtensorMap* map, void* base, int64_t rows, int64_t cols, int64_t ld) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return W4A4_ERR_CUDA;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld * 2)};
+  const cuuint32_t box[2] = {32u, 32u};
+  const cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? W4A4_OK : W4A4_ERR_CUDA;
+}
+
 inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 inline size_t round256(size_t b) { return (b + 255) / 256 * 256; }
 
@@ -156,9 +171,14 @@ int run_linear(const int8_t* Xq, const float* sx, const int8_t* Wq, const float*
     a.status = dev->status;
     return smallm_launch_tm(tmW, tmX, a, dev->num_sms, stream) == cudaSuccess ? W4A4_OK : W4A4_ERR_CUDA;
   }
-  CUtensorMap tmA, tmB;
+  CUtensorMap tmA, tmB, tmY;
   if ((st = packed_map(&tmA, Xq, M, K, kGemmBM / 2)) != W4A4_OK) return st;
   if ((st = packed_map(&tmB, Wq, N, K, kGemmBN / 2)) != W4A4_OK) return st;
+  if (out_s32) {
+    tmY = tmA;   // not read by the int32 epilogue
+  } else if ((st = output_map(&tmY, out, M, N, ldo)) != W4A4_OK) {
+    return st;
+  }
   GemmArgs a{};
   a.M = M;
   a.N = N;
@@ -170,7 +190,7 @@ int run_linear(const int8_t* Xq, const float* sx, const int8_t* Wq, const float*
   a.ldo = ldo;
   a.out_s32 = out_s32;
   a.status = dev->status;
-  return gemm_tc_launch(tmA, tmB, a, dev->num_sms, stream) == cudaSuccess ? W4A4_OK : W4A4_ERR_CUDA;
+  return gemm_tc_launch(tmA, tmB, tmY, a, dev->num_sms, stream) == cudaSuccess ? W4A4_OK : W4A4_ERR_CUDA;
 }
 
 __global__ void wait_forever_bounded_kernel(unsigned long long limit_ns, unsigned int* status) {

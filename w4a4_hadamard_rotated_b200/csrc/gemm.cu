@@ -29,9 +29,13 @@
 //   * One thread of the even CTA issues the MMAs; tcgen05.commit with a
 //     cluster multicast frees a ring slot in both CTAs at once.  The
 //     accumulator is double-buffered in tensor memory (2 x 256 columns), so
-//     four epilogue warps per CTA drain tile i (tcgen05.ld, y = bf16(((float)acc
-//     * sx[m]) * sw[n] + bias[n]) with explicitly rounded fp32 steps) while the
-//     MMAs of tile i+1 run.
+//     four epilogue warps per CTA drain tile i while the MMAs of tile i+1 run:
+//     the tile's column scales and bias are staged once in shared memory, the
+//     tcgen05.ld of the next 32 columns is in flight while the current ones
+//     are converted, and y = bf16(((float)acc * sx[m]) * sw[n] + bias[n]) is
+//     formed with separately rounded fp32 steps (paired .f32x2 arithmetic);
+//     each 32 x 32 bf16 block is staged in shared memory (64-byte swizzle)
+//     and written with one TMA tensor store, which also clips the M/N tails.
 //   * The kernel is persistent: the clusters walk the tiles with a static
 //     stride.  Every wait is bounded: an expired wait records W4A4_ERR_TIMEOUT
 //     in the device status word, every role stops, the MMAs are drained and
@@ -55,13 +59,21 @@ constexpr int BK = 128;         // int4 codes per k-block (= bytes per widened r
 constexpr int BKP = BK / 2;     // packed bytes per row per k-block
 constexpr int SP = 4;           // packed ring depth
 constexpr int SWD = 4;          // widened ring depth
-constexpr int kWidenWarps = 8;
+// Warp roles.  A warp runs on SM sub-partition (warp % 4).  The threads that
+// issue tcgen05.mma and TMA instructions hold their sub-partition's issue
+// slot for long stretches, so they share sub-partition 0 with one epilogue
+// warp and no widen warp; the nine widen warps sit three to a sub-partition on
+// 1..3, next to one epilogue warp each (an epilogue warp may only read the
+// tensor-memory lane quarter warp % 4).
+constexpr int kWidenWarps = 9;
 constexpr int kEpiWarps = 4;
 constexpr int kWarpMma = 0;
-constexpr int kWarpTma = 1;
-constexpr int kWarpWiden0 = 2;
-constexpr int kWarpEpi0 = kWarpWiden0 + kWidenWarps;
-constexpr int kThreads = (kWarpEpi0 + kEpiWarps) * 32;
+constexpr int kWarpTma = 4;
+constexpr int kThreads = 16 * 32;
+__device__ __forceinline__ bool is_epi_warp(int w) { return w == 8 || w >= 13; }
+__device__ __forceinline__ bool is_widen_warp(int w) { return w != 0 && w != 4 && w != 8 && w < 12; }
+// widen warps 1,2,3,5,6,7,9,10,11 -> 0..8
+__device__ __forceinline__ int widen_index(int w) { return w - 1 - (w > 4) - (w > 8); }
 constexpr int kTmemCols = 2 * BN;   // two int32 accumulators of BN columns
 
 constexpr uint32_t kWideA = HM * BK;     // 16 KB
@@ -71,12 +83,17 @@ constexpr uint32_t kPackA = HM * BKP;    // 8 KB
 constexpr uint32_t kPackB = HN * BKP;    // 8 KB
 constexpr uint32_t kPStage = kPackA + kPackB;
 constexpr uint32_t kOffPack = SWD * kStage;
-constexpr uint32_t kSmemBytes = kOffPack + SP * kPStage;
+// epilogue staging: per epilogue warp two 32 x 32 bf16 boxes (64-byte rows,
+// 64-byte swizzle) for the TMA stores of y
+constexpr uint32_t kStageBox = 32 * 64;
+constexpr uint32_t kOffEpi = kOffPack + SP * kPStage;
+constexpr uint32_t kSmemBytes = kOffEpi + 4 * 2 * kStageBox;
 constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;   // slack for 1024-byte alignment
 
 // packed 16-byte units per CTA and k-block: (HM + HN) rows x 4 units
 constexpr int kUnits = (HM + HN) * (BKP / 16);
-constexpr int kUnitsPerThread = kUnits / (kWidenWarps * 32);   // 4
+constexpr int kWidenThreads = kWidenWarps * 32;
+constexpr int kUnitsPerThread = (kUnits + kWidenThreads - 1) / kWidenThreads;   // 4 (the last partly idle)
 
 struct Bars {
   uint64_t packed_full[SP];   // TMA transaction barrier
@@ -92,6 +109,26 @@ struct Bars {
   int abort_flag;
 };
 
+// Packed fp32 pairs (sm_100 .f32x2 arithmetic) for the epilogue.
+__device__ __forceinline__ uint64_t pk2(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void upk2(uint64_t r, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
 // Widening without sign extension: a signed nibble q placed in the high half
 // of a byte IS the signed byte 16*q.  The nibbles of a 32-bit word go to bytes
 // in the order (1,3,5,7, 0,2,4,6); that K permutation is the same for both
@@ -106,11 +143,14 @@ __device__ __forceinline__ void widen_word16(uint32_t w, uint32_t& o0, uint32_t&
 __device__ __forceinline__ void widen_units(const uint8_t* __restrict__ pstage, uint8_t* __restrict__ stage, int wt) {
   uint4 buf[kUnitsPerThread];
 #pragma unroll
-  for (int i = 0; i < kUnitsPerThread; ++i)
-    buf[i] = *reinterpret_cast<const uint4*>(pstage + (wt + i * kWidenWarps * 32) * 16);
+  for (int i = 0; i < kUnitsPerThread; ++i) {
+    const int u = wt + i * kWidenThreads;
+    if (u < kUnits) buf[i] = *reinterpret_cast<const uint4*>(pstage + u * 16);
+  }
 #pragma unroll
   for (int i = 0; i < kUnitsPerThread; ++i) {
-    const int u = wt + i * kWidenWarps * 32;
+    const int u = wt + i * kWidenThreads;
+    if (u >= kUnits) break;
     const bool isA = u < HM * 4;
     const int uu = isA ? u : u - HM * 4;
     const int r = uu >> 2;
@@ -129,9 +169,12 @@ __device__ __forceinline__ void widen_units(const uint8_t* __restrict__ pstage, 
 
 template <int OUT_S32>
 __global__ void __launch_bounds__(kThreads, 1)
-    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmArgs args) {
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ CUtensorMap tmY, GemmArgs args) {
   extern __shared__ uint8_t smem_dyn[];
   __shared__ Bars bars;
+  __shared__ __align__(16) float epi_sw[2][BN];
+  __shared__ __align__(16) float epi_bias[2][BN];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
 
   const int warp = threadIdx.x >> 5;
@@ -211,16 +254,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       (void)mbar_wait_cluster(&bars.drain, 0, nullptr, nullptr, 100000000ull);
     } else if (rank == 1 && lane == 0) {
       // Forwarder: a completed ring slot of this (odd) CTA becomes one arrival
-      // on the even CTA's barrier.  The widen warps only release locally (a
-      // cluster-scope release would wait for their prefetch loads in flight);
-      // this thread has no memory traffic of its own, and it forwards in the
-      // order the MMA consumes the slots.
+      // on the even CTA's barrier, published with a release fence restricted
+      // to shared memory and a relaxed cluster arrive (a full cluster-scope
+      // release costs about a microsecond).  The widen warps only release
+      // locally; this thread forwards in the order the MMA consumes the slots.
       uint32_t ws = 0, wph = 0;
       for (int t = cluster; t < tiles; t += nclusters) {
         bool ok = true;
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait(&bars.wide_full[ws], wph, abort_flag, args.status)) { ok = false; break; }
-          mbar_arrive_remote(&bars.wide_full[ws], 0);
+          mbar_arrive_remote_smem(&bars.wide_full[ws], 0);
           if (++ws == SWD) { ws = 0; wph ^= 1; }
         }
         if (!ok) break;
@@ -252,9 +295,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else if (warp < kWarpEpi0) {
+  } else if (is_widen_warp(warp)) {
     // ------------------------------------------------------------ widen warps
-    const int wt = threadIdx.x - kWarpWiden0 * 32;
+    const int wt = widen_index(warp) * 32 + lane;
     uint32_t ps = 0, ph = 0, ws = 0, wph = 0;
     bool ok = true;
     for (int t = cluster; t < tiles && ok; t += nclusters) {
@@ -272,99 +315,113 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (++ws == SWD) { ws = 0; wph ^= 1; }
       }
     }
-  } else {
+  } else if (is_epi_warp(warp)) {
     // ------------------------------------------------------------ epilogue warps
     const int q = warp & 3;   // TMEM lane quarter this warp may access
+    const int et = q * 32 + lane;   // 0..127 across the four epilogue warps
+    uint8_t* epi_stage = smem + kOffEpi + q * 2 * kStageBox;
     uint32_t acc_ph = 0;
     int lt = 0;
     for (int t = cluster; t < tiles; t += nclusters, ++lt) {
       const int ab = lt & 1;
       const int mb = t % num_m, nb = t / num_m;
-      if (!warp_wait_cluster(&bars.acc_full[ab], (acc_ph >> ab) & 1, abort_flag, args.status)) break;
+      const int64_t nt0 = static_cast<int64_t>(nb) * BN;
+      // the tile's column scales and bias, staged once (double-buffered by tile)
+      float* sws = epi_sw[ab];
+      float* bs = epi_bias[ab];
+      if (!OUT_S32) {
+#pragma unroll
+        for (int j = et; j < BN; j += 128) {
+          const int64_t n = nt0 + j;
+          sws[j] = n < N ? args.sw[n] : 0.0f;
+          bs[j] = (n < N && args.bias != nullptr) ? __uint_as_float(static_cast<uint32_t>(args.bias[n]) << 16) : 0.0f;
+        }
+      }
+      (void)warp_wait_cluster(&bars.acc_full[ab], (acc_ph >> ab) & 1, abort_flag, args.status);
       acc_ph ^= 1u << ab;
+      // staged scales visible to the four warps; every wait above is bounded, so
+      // all four always arrive here and then leave together on an abort
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (*abort_flag) break;
       tc_fence_after();
       const int64_t m = static_cast<int64_t>(mb) * BM + rank * HM + q * 32 + lane;
       const bool mrow = m < M;
       float sxm = 0.0f;
       if (!OUT_S32 && mrow) sxm = args.sx[m];
-#pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t r[32];
-        __syncwarp();
-        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + ab * BN + c * 32, r);
-        tmem_wait_ld();
+      const uint64_t sx2 = pk2(sxm, sxm);
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + ab * BN;
+      uint32_t r[2][32];
+      tmem_ld_32x32b_x32(tbase, r[0]);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) r[i] = static_cast<uint32_t>(static_cast<int32_t>(r[i]) >> 8);
-        const int64_t n0 = static_cast<int64_t>(nb) * BN + c * 32;
-        if (!mrow || n0 >= N) continue;   // the loads above stay warp-uniform
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t (&cur)[32] = r[c & 1];
+        tmem_wait_ld();
+        // the next chunk's tensor-memory load overlaps this chunk's math
+        if (c + 1 < BN / 32) tmem_ld_32x32b_x32(tbase + (c + 1) * 32, r[(c + 1) & 1]);
+        const int64_t n0 = nt0 + c * 32;
+        if (n0 >= N) continue;   // warp-uniform; the tensor-memory loads above stay aligned
         const bool full = n0 + 32 <= N;
         if (OUT_S32) {
+          if (!mrow) continue;
+          int32_t v[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = static_cast<int32_t>(cur[i]) >> 8;
           int32_t* dst = reinterpret_cast<int32_t*>(args.out) + m * args.ldo + n0;
           if (full) {
 #pragma unroll
             for (int i = 0; i < 8; ++i)
-              reinterpret_cast<uint4*>(dst)[i] = make_uint4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
+              reinterpret_cast<int4*>(dst)[i] = make_int4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
           } else {
 #pragma unroll
             for (int i = 0; i < 32; ++i)
-              if (n0 + i < N) dst[i] = static_cast<int32_t>(r[i]);
+              if (n0 + i < N) dst[i] = v[i];
           }
         } else {
-          uint16_t* dst = reinterpret_cast<uint16_t*>(args.out) + m * args.ldo + n0;
-          float swv[32], bv[32];
-          if (full) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const float4 s4 = __ldg(reinterpret_cast<const float4*>(args.sw + n0) + i);
-              swv[4 * i] = s4.x; swv[4 * i + 1] = s4.y; swv[4 * i + 2] = s4.z; swv[4 * i + 3] = s4.w;
-            }
-            if (args.bias != nullptr) {
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const uint4 b4 = __ldg(reinterpret_cast<const uint4*>(args.bias + n0) + i);
-                const uint32_t bw[4] = {b4.x, b4.y, b4.z, b4.w};
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                  bv[8 * i + 2 * j] = __uint_as_float(bw[j] << 16);
-                  bv[8 * i + 2 * j + 1] = __uint_as_float(bw[j] & 0xFFFF0000u);
-                }
-              }
-            }
-          } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const bool in = n0 + i < N;
-              swv[i] = in ? args.sw[n0 + i] : 0.0f;
-              bv[i] = (in && args.bias != nullptr) ? __uint_as_float(static_cast<uint32_t>(args.bias[n0 + i]) << 16) : 0.0f;
-            }
-          }
           uint32_t packed[16];
+          const float* swc = sws + c * 32;
+          const float* bc = bs + c * 32;
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            float y0 = __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(r[2 * i])), sxm), swv[2 * i]);
-            float y1 = __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(r[2 * i + 1])), sxm), swv[2 * i + 1]);
+            // ((float)acc * sx) * sw (+ bias), each step rounded on its own
+            const uint64_t a2 = pk2(__int2float_rn(static_cast<int32_t>(cur[2 * i]) >> 8),
+                                    __int2float_rn(static_cast<int32_t>(cur[2 * i + 1]) >> 8));
+            const float2 w2 = *reinterpret_cast<const float2*>(swc + 2 * i);
+            uint64_t y2 = mul2(mul2(a2, sx2), pk2(w2.x, w2.y));
             if (args.bias != nullptr) {
-              y0 = __fadd_rn(y0, bv[2 * i]);
-              y1 = __fadd_rn(y1, bv[2 * i + 1]);
+              const float2 b2 = *reinterpret_cast<const float2*>(bc + 2 * i);
+              y2 = add2(y2, pk2(b2.x, b2.y));
             }
+            float y0, y1;
+            upk2(y2, y0, y1);
             const __nv_bfloat162 h = __floats2bfloat162_rn(y0, y1);
             packed[i] = *reinterpret_cast<const uint32_t*>(&h);
           }
-          if (full) {
+          // stage the 32 x 32 block (row = lane, 64-byte swizzle: chunk j of
+          // row r at chunk j ^ ((r >> 1) & 3); conflict-free for this pattern)
+          uint8_t* box = epi_stage + ((c & 1) * kStageBox);
+          // the store that last used this box (two chunks ago, possibly in the
+          // previous tile) must have finished reading it
+          if (lane == 0) bulk_wait_group_read<1>();
+          __syncwarp();
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-              reinterpret_cast<uint4*>(dst)[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
-          } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (n0 + i < N) dst[i] = static_cast<uint16_t>((packed[i >> 1] >> (16 * (i & 1))) & 0xFFFFu);
+          for (int j = 0; j < 4; ++j)
+            *reinterpret_cast<uint4*>(box + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4)) =
+                make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+          fence_async_shared();
+          __syncwarp();
+          // a box whose first row is past M stores nothing (rows past M inside
+          // a box are clipped by the tensor map)
+          if (lane == 0 && m < M) {
+            tma_store_2d(&tmY, box, static_cast<int32_t>(n0), static_cast<int32_t>(m));
+            bulk_commit_group();
           }
         }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_remote(&bars.acc_empty[ab], 0);
+      if (lane == 0) mbar_arrive_remote_smem(&bars.acc_empty[ab], 0);
     }
+    if (lane == 0) bulk_wait_group<0>();   // every store of y has completed
   }
 
   tc_fence_before();
@@ -406,8 +463,8 @@ int max_clusters(int num_sms) {
 }
 
 template <int OUT_S32>
-cudaError_t launch(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a, int64_t tiles, int num_sms,
-                   cudaStream_t stream) {
+cudaError_t launch(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmY, const GemmArgs& a,
+                   int64_t tiles, int num_sms, cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<OUT_S32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(kSmemAlloc));
   if (e != cudaSuccess) return e;
@@ -425,17 +482,17 @@ cudaError_t launch(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArg
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<OUT_S32>, tmA, tmB, a);
+  return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<OUT_S32>, tmA, tmB, tmY, a);
 }
 
 }  // namespace
 
-cudaError_t gemm_tc_launch(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a, int num_sms,
-                           cudaStream_t stream) {
+cudaError_t gemm_tc_launch(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmY, const GemmArgs& a,
+                           int num_sms, cudaStream_t stream) {
   const int64_t tiles = ((a.M + BM - 1) / BM) * ((a.N + BN - 1) / BN);
   if (tiles == 0) return cudaSuccess;
   cudaError_t e =
-      a.out_s32 ? launch<1>(tmA, tmB, a, tiles, num_sms, stream) : launch<0>(tmA, tmB, a, tiles, num_sms, stream);
+      a.out_s32 ? launch<1>(tmA, tmB, tmY, a, tiles, num_sms, stream) : launch<0>(tmA, tmB, tmY, a, tiles, num_sms, stream);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

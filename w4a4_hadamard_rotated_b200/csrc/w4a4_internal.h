@@ -32,9 +32,11 @@ struct GemmArgs {
   unsigned int* status;   // device status word (bounded-wait timeouts)
 };
 // tmA: packed activations [M, K/2] bytes, tmB: packed weights [N, K/2] bytes,
-// both with box {64 bytes, kGemmBM/2 rows}.  Launched as clusters of 2 CTAs.
-cudaError_t gemm_tc_launch(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a, int num_sms,
-                           cudaStream_t stream);
+// both with box {64 bytes, kGemmBM/2 rows}; tmY: bf16 output [M, N] (row
+// stride ldo) with box {32, 32} and 64-byte swizzle (unused for int32 output).
+// Launched as clusters of 2 CTAs.
+cudaError_t gemm_tc_launch(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmY, const GemmArgs& a,
+                           int num_sms, cudaStream_t stream);
 constexpr int kGemmBM = 256;
 constexpr int kGemmBN = 256;
 
