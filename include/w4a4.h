@@ -63,7 +63,7 @@ int w4a4_version(void);
  * int4 pairs (low-nibble-first, [N, K/2] int8 container) with fp32 [N, 1]
  * per-row scales".
  *   W   [N, K] fp32, row stride ldw >= K (elements), 16-byte aligned, ldw % 4 == 0
- *   N >= 1;  K % 128 == 0, K % g == 0, 128 <= K <= 65536;  g in {64,128,256}
+ *   N >= 1;  K % 128 == 0, K % g == 0, 128 <= K <= 24576;  g in {64,128,256}
  *   Wq  [N, K/2] int8 output, contiguous rows, 16-byte aligned
  *   sw  [N] fp32 output
  */
@@ -77,7 +77,7 @@ int w4a4_quantize_weight(const float* W, int64_t N, int64_t K, int64_t ldw, int 
  *   act 0: none; 1: exact-erf GELU applied to x before the rotation (used to
  *       feed an MLP down projection from the up projection's output)
  *   Xq  [M, K/2] int8 output (contiguous rows, 16-byte aligned); sx [M] fp32
- *   M >= 0 (M == 0 is a no-op); K and g as for w4a4_quantize_weight.
+ *   M >= 0 (M == 0 is a no-op); K % 128 == 0, K % g == 0, 128 <= K <= 32768.
  * A row that is all zero gets sx = 0 and all-zero codes.
  */
 int w4a4_quantize_activation(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int g,
@@ -91,10 +91,12 @@ int w4a4_quantize_activation(const uint16_t* x, int64_t M, int64_t K, int64_t ld
  *   Wq [N, K/2] int8, sw [N] fp32 (from w4a4_quantize_weight)
  *   bias [N] bf16 bits or NULL
  *   y  [M, N] bf16 bits output, row stride ldy >= N, ldy % 8 == 0, 16-byte aligned
- *   M >= 0, N >= 1, N % 8 == 0, K >= 32, K % 32 == 0; Xq/Wq 16-byte aligned
+ *   M >= 0, N >= 1, N % 8 == 0, 32 <= K <= 131072, K % 32 == 0; Xq/Wq 16-byte aligned
  *   workspace: device scratch of at least w4a4_workspace_bytes(M, N, K)
- *       bytes, 256-byte aligned (may be NULL when that size is 0).  Calls that
- *       share one workspace must be ordered on the same stream.
+ *       bytes, 256-byte aligned (may be NULL when that size is 0).  Its first
+ *       32 KiB (arrival counters of the small-M kernel) must be zero before the
+ *       first call; every call leaves them zero.  Calls that share one
+ *       workspace must be ordered on the same stream.
  * M <= 64 takes the weight-streaming split-K kernel, larger M the tcgen05
  * tensor-core kernel; both give bit-identical int32 accumulators.
  */
@@ -106,7 +108,10 @@ int w4a4_linear(const int8_t* Xq, const float* sx, const int8_t* Wq, const float
  * Fused layer: w4a4_quantize_activation followed by w4a4_linear, with the
  * packed activation and its scales kept in the workspace.
  *   x [M, K] bf16 bits with row stride ldx; other arguments as above.
- *   workspace: at least w4a4_fused_workspace_bytes(M, N, K) bytes.
+ *   workspace: at least w4a4_fused_workspace_bytes(M, N, K) bytes, laid out as
+ *       [small-M scratch, counter block first][packed x][sx]; the same rule for
+ *       its first 32 KiB holds, so one zero-filled buffer can serve both
+ *       w4a4_linear and w4a4_linear_fused calls of any shape.
  */
 int w4a4_linear_fused(const uint16_t* x, int64_t ldx, const int8_t* Wq, const float* sw,
                       const uint16_t* bias, uint16_t* y, int64_t ldy, int64_t M, int64_t N,
