@@ -16,7 +16,8 @@
  *
  * Conventions for every entry point:
  *   - Every tensor pointer is DEVICE memory owned by the caller; the library
- *     never allocates or frees memory.  Matrices are row-major with the
+ *     never allocates or frees memory (w4a4_linear_noalloc uses a fixed array
+ *     of the library's own device memory instead of a caller workspace).  Matrices are row-major with the
  *     inner dimension contiguous; ld* arguments are row strides in elements.
  *   - bf16 tensors are passed as raw 16-bit patterns (uint16_t).
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  All work is
@@ -132,6 +133,31 @@ size_t w4a4_fused_workspace_bytes(int64_t M, int64_t N, int64_t K);
 int w4a4_gemm_s32(const int8_t* Xq, const int8_t* Wq, int32_t* acc, int64_t M, int64_t N,
                   int64_t K, int64_t ldc, int path, void* workspace, size_t workspace_bytes,
                   void* stream);
+
+/*
+ * Small-M W4A4 linear (1 <= M <= 64) that allocates nothing and takes no
+ * workspace.  The pages have no counterpart to this entry point; it exists
+ * for callers that cannot allocate device memory when they run the layer --
+ * for instance a plug-in whose host framework owns every byte of device
+ * memory and hands a custom op no scratch, or a latency-critical decode loop
+ * that must not call cudaMalloc after start-up (an allocation can
+ * synchronise the device and fragment a pool sized in advance).
+ *   Arguments, layouts and results are those of w4a4_linear; the output is
+ *   bit-identical to it.  Scratch (split-K partial tiles and arrival
+ *   counters) lives in a fixed 4 MiB array of this library's own device
+ *   memory, which every GPU that loads the library keeps until the process
+ *   exits; a shape whose scratch, w4a4_workspace_bytes(M, N, K), exceeds
+ *   4 MiB is rejected with W4A4_ERR_WORKSPACE before anything is launched
+ *   (M > 64 or N > 1048576 gives W4A4_ERR_SHAPE).
+ *   The first call on a device resolves the array's device address and
+ *   clears its counter block on `stream`; make that first call before any
+ *   stream capture.  Every call uses the same array and leaves the counters
+ *   at zero; calls that may overlap on the GPU (other streams, other host
+ *   threads) race on the array and must be serialised by the caller.
+ */
+int w4a4_linear_noalloc(const int8_t* Xq, const float* sx, const int8_t* Wq, const float* sw,
+                        const uint16_t* bias, uint16_t* y, int64_t M, int64_t N, int64_t K, int64_t ldy,
+                        void* stream);
 
 /*
  * Synchronise `stream`, then read and clear the device status word that

@@ -43,6 +43,7 @@ SIGNATURES = {
     "w4a4_workspace_bytes": (_SZ, [_I64, _I64, _I64]),
     "w4a4_fused_workspace_bytes": (_SZ, [_I64, _I64, _I64]),
     "w4a4_gemm_s32": (_I, [_P, _P, _P, _I64, _I64, _I64, _I64, _I, _P, _SZ, _P]),
+    "w4a4_linear_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P]),
     "w4a4_last_device_error": (_I, [_P]),
     "w4a4_debug_wait_timeout": (_I, [_I64, _P]),
 }
@@ -193,6 +194,20 @@ def gemm_s32(Xq, Wq, path=0, out=None):
     _check(lib.w4a4_gemm_s32(_ptr(Xq), _ptr(Wq), _ptr(acc), M, N, K, acc.stride(0), path, _ptr(ws), nbytes,
                              _stream(Xq)), "w4a4_gemm_s32")
     return acc
+
+
+def linear_noalloc(Xq, sx, Wq, sw, bias=None, out=None):
+    """Small-M (M <= 64) linear with no workspace: the library's own fixed
+    scratch array stands in for it (see w4a4_linear_noalloc in the header)."""
+    lib = load_library()
+    _need_cuda(Xq, torch.int8, "Xq")
+    _need_cuda(Wq, torch.int8, "Wq")
+    M, Kh = Xq.shape
+    N = Wq.shape[0]
+    y = out if out is not None else torch.empty(M, N, dtype=torch.bfloat16, device=Xq.device)
+    _check(lib.w4a4_linear_noalloc(_ptr(Xq), _ptr(sx), _ptr(Wq), _ptr(sw), _ptr(bias), _ptr(y), M, N, 2 * Kh,
+                                   y.stride(0), _stream(Xq)), "w4a4_linear_noalloc")
+    return y
 
 
 def last_device_error(device=None):

@@ -19,16 +19,10 @@ namespace w4a4 {
 __device__ unsigned int g_device_status = 0;
 
 namespace {
-
 constexpr int kMaxDevices = 64;
-
-struct DeviceInfo {
-  int checked = 0;     // 0 unknown, 1 supported, -1 unsupported
-  int num_sms = 0;
-  unsigned int* status = nullptr;
-};
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
+}  // namespace
 
 // Resolve the current device; fills its SM count and the device address of
 // the status word on first use.
@@ -59,6 +53,8 @@ int current_device(DeviceInfo** out) {
   return W4A4_OK;
 }
 
+namespace {
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -76,6 +72,8 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+}  // namespace
+
 // 2-D map over a packed int4 matrix [rows, K/2] bytes, box {64 bytes, box_rows};
 // out-of-range rows and columns read as zero.
 int packed_map(CUtensorMap* map, const int8_t* base, int64_t rows, int64_t K, int box_rows) {
@@ -90,6 +88,8 @@ int packed_map(CUtensorMap* map, const int8_t* base, int64_t rows, int64_t K, in
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? W4A4_OK : W4A4_ERR_CUDA;
 }
+
+namespace {
 
 // 2-D map over a bf16 output [rows, cols] with row stride ld (elements), box
 // {32, 32}, 64-byte swizzle (the epilogue's staging layout).
@@ -206,6 +206,26 @@ __global__ void wait_forever_bounded_kernel(unsigned long long limit_ns, unsigne
 }
 
 }  // namespace
+
+int validate_linear(const int8_t* Xq, const float* sx, const int8_t* Wq, const float* sw,
+                           const uint16_t* bias, const void* y, int64_t M, int64_t N, int64_t K, int64_t ldy,
+                           int out_s32) {
+  if (Wq == nullptr || (!out_s32 && sw == nullptr)) return W4A4_ERR_NULL;
+  // an empty batch (M == 0) may pass NULL for its zero-size tensors
+  if (M != 0 && (Xq == nullptr || y == nullptr || (!out_s32 && sx == nullptr))) return W4A4_ERR_NULL;
+  int st = check_gemm_shape(M, N, K);
+  if (st != W4A4_OK) return st;
+  if (ldy < N) return W4A4_ERR_SHAPE;
+  if (!aligned(Xq, 16) || !aligned(Wq, 16) || !aligned(y, 16)) return W4A4_ERR_ALIGN;
+  if (out_s32) {
+    if (ldy % 4 != 0) return W4A4_ERR_ALIGN;
+  } else {
+    if (ldy % 8 != 0 || !aligned(sw, 16) || !aligned(sx, 4)) return W4A4_ERR_ALIGN;
+    if (bias != nullptr && !aligned(bias, 16)) return W4A4_ERR_ALIGN;
+  }
+  return W4A4_OK;
+}
+
 }  // namespace w4a4
 
 using namespace w4a4;
@@ -284,25 +304,6 @@ size_t w4a4_fused_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   if (M <= 0 || N <= 0 || K <= 0) return 0;
   return fused_linear_part(M, N, K) + round256(static_cast<size_t>(M) * static_cast<size_t>(K / 2)) +
          round256(static_cast<size_t>(M) * 4);
-}
-
-static int validate_linear(const int8_t* Xq, const float* sx, const int8_t* Wq, const float* sw,
-                           const uint16_t* bias, const void* y, int64_t M, int64_t N, int64_t K, int64_t ldy,
-                           int out_s32) {
-  if (Wq == nullptr || (!out_s32 && sw == nullptr)) return W4A4_ERR_NULL;
-  // an empty batch (M == 0) may pass NULL for its zero-size tensors
-  if (M != 0 && (Xq == nullptr || y == nullptr || (!out_s32 && sx == nullptr))) return W4A4_ERR_NULL;
-  int st = check_gemm_shape(M, N, K);
-  if (st != W4A4_OK) return st;
-  if (ldy < N) return W4A4_ERR_SHAPE;
-  if (!aligned(Xq, 16) || !aligned(Wq, 16) || !aligned(y, 16)) return W4A4_ERR_ALIGN;
-  if (out_s32) {
-    if (ldy % 4 != 0) return W4A4_ERR_ALIGN;
-  } else {
-    if (ldy % 8 != 0 || !aligned(sw, 16) || !aligned(sx, 4)) return W4A4_ERR_ALIGN;
-    if (bias != nullptr && !aligned(bias, 16)) return W4A4_ERR_ALIGN;
-  }
-  return W4A4_OK;
 }
 
 int w4a4_linear(const int8_t* Xq, const float* sx, const int8_t* Wq, const float* sw, const uint16_t* bias,

@@ -364,3 +364,80 @@ cudaError_t smallm_launch_tm(const CUtensorMap& tmW, const CUtensorMap& tmX, con
 int smallm_rows_padded(int64_t M) { return M <= 16 ? 16 : (M <= 32 ? 32 : 64); }
 
 }  // namespace w4a4
+
+// ---------------------------------------------------------------------------
+// Small-M linear that allocates nothing (w4a4_linear_noalloc in w4a4.h).
+//
+// Same kernel and launch as the workspace-taking path; only the scratch is
+// different: the arrival counters and split-K slots live in a fixed array of
+// this library's own device memory instead of a caller workspace.
+// ---------------------------------------------------------------------------
+#include <mutex>
+
+#include "w4a4.h"
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;   // 4 MiB: counter block + split-K slots
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kNoAllocMaxDevices = 64;
+void* g_noalloc_ptr[kNoAllocMaxDevices] = {nullptr};   // device address of the array, per device
+std::mutex g_noalloc_mu;
+
+// Device address of the scratch array on the current device.  The host-side
+// name g_noalloc_scratch is only a stand-in for the symbol, never a device
+// pointer, so its address is resolved once per device with
+// cudaGetSymbolAddress (with that device current) and cached; the same first
+// call clears the counter block on `stream` (the counters must start at zero;
+// every completed call leaves them at zero again).
+int noalloc_scratch(uint8_t** out, cudaStream_t stream) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return W4A4_ERR_CUDA;
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return W4A4_ERR_DEVICE;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return W4A4_ERR_CUDA;
+    if (cudaMemsetAsync(p, 0, w4a4::kSmallMCounterBytes, stream) != cudaSuccess) return W4A4_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = static_cast<uint8_t*>(g_noalloc_ptr[dev]);
+  return W4A4_OK;
+}
+
+}  // namespace
+
+extern "C" int w4a4_linear_noalloc(const int8_t* Xq, const float* sx, const int8_t* Wq, const float* sw,
+                                   const uint16_t* bias, uint16_t* y, int64_t M, int64_t N, int64_t K, int64_t ldy,
+                                   void* stream) {
+  using namespace w4a4;
+  int st = validate_linear(Xq, sx, Wq, sw, bias, y, M, N, K, ldy, 0);
+  if (st != W4A4_OK) return st;
+  if (M < 1 || M > kSmallMMax || N > kSmallMMaxN) return W4A4_ERR_SHAPE;
+  if (smallm_workspace_bytes(M, N, K) > kNoAllocScratchBytes) return W4A4_ERR_WORKSPACE;
+  DeviceInfo* dev = nullptr;
+  if ((st = current_device(&dev)) != W4A4_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* scratch = nullptr;
+  if ((st = noalloc_scratch(&scratch, s)) != W4A4_OK) return st;
+  CUtensorMap tmW, tmX;
+  if ((st = packed_map(&tmW, Wq, N, K, WM)) != W4A4_OK) return st;
+  if ((st = packed_map(&tmX, Xq, M, K, smallm_rows_padded(M))) != W4A4_OK) return st;
+  SmallMArgs a{};
+  a.xq = Xq;
+  a.wq = Wq;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.sx = sx;
+  a.sw = sw;
+  a.bias = bias;
+  a.out = y;
+  a.ldo = ldy;
+  a.out_s32 = 0;
+  a.counters = reinterpret_cast<unsigned int*>(scratch);
+  a.partial = reinterpret_cast<int32_t*>(scratch + kSmallMCounterBytes);
+  a.status = dev->status;
+  return smallm_launch_tm(tmW, tmX, a, dev->num_sms, s) == cudaSuccess ? W4A4_OK : W4A4_ERR_CUDA;
+}

@@ -9,6 +9,20 @@
 
 namespace w4a4 {
 
+// ---- shared host helpers (api.cu)
+struct DeviceInfo {
+  int checked = 0;     // 0 unknown, 1 supported, -1 unsupported
+  int num_sms = 0;
+  unsigned int* status = nullptr;   // device address of the status word
+};
+// The current device (must be sm_100); W4A4_OK or an error status.
+int current_device(DeviceInfo** out);
+// TMA map over a packed int4 matrix [rows, K/2] bytes with box {64, box_rows}.
+int packed_map(CUtensorMap* map, const int8_t* base, int64_t rows, int64_t K, int box_rows);
+// Argument checks of w4a4_linear (out_s32 = 0) / w4a4_gemm_s32 (out_s32 = 1).
+int validate_linear(const int8_t* Xq, const float* sx, const int8_t* Wq, const float* sw, const uint16_t* bias,
+                    const void* y, int64_t M, int64_t N, int64_t K, int64_t ldy, int out_s32);
+
 // ---- activation / weight rotate + quantise + pack (quant.cu)
 cudaError_t rotate_quant_bf16(const uint16_t* x, int64_t M, int K, int64_t ldx, int g, int act, int8_t* out,
                               float* scale, int num_sms, unsigned int* status, cudaStream_t stream);
