@@ -14,7 +14,6 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
 import sys
 import threading
 import time
@@ -30,6 +29,10 @@ PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 INT8_OVER_BF16 = 2.0      # nominal dense int8 : bf16 tensor throughput on B200 (4.5 : 2.25 PFLOP/s)
 N_SETS = 5
+# DRAM bytes (read + write) per launch from ncu captures of the current
+# kernels, keyed by (kernel, workload); a kernel that changed since its
+# capture has no entry (traffic reported as null).  Figures: profiles/.
+MEASURED_TRAFFIC = {}
 
 
 def load_peaks():
@@ -41,57 +44,60 @@ def load_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle sampling in the background."""
+    """Samples SM clocks and throttle reasons during the timed region: NVML
+    polled every 10 ms from a thread."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4}
 
     def __init__(self, device_index):
         self.dev = device_index
-        self.proc = None
-        self.lines = []
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
 
     def start(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100", "-i", str(self.dev)],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
-            self.thread.start()
-        except (OSError, ValueError):
-            self.proc = None
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByIndex(self._nvml_index())
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            def run():
+                while not self._stop.is_set():
+                    try:
+                        self.samples.append(float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)))
+                        mask = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                        for name, bit in self.REASONS.items():
+                            if mask & bit:
+                                self.reasons.add(name)
+                    except Exception:
+                        pass
+                    time.sleep(0.01)
+
+            self._thread = threading.Thread(target=run, daemon=True)
+            self._thread.start()
+        except Exception:
+            self._thread = None
+
+    def _nvml_index(self):
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        if vis:
+            try:
+                return int(vis.split(",")[self.dev])
+            except (ValueError, IndexError):
+                pass
+        return self.dev
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        self.thread.join(timeout=2)
-        sm, smax, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                smax = float(parts[2])
-            except ValueError:
-                continue
-            for nm, val in zip(names, parts[5:9]):
-                if val.lower() == "active":
-                    reasons.add(nm)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        if self._thread is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"], "samples": 0}
+        self._stop.set()
+        self._thread.join(timeout=2)
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
 def dist_setup():
@@ -186,20 +192,44 @@ def run_reference(args, cfg, world, rank):
     print(json.dumps(line), flush=True)
 
 
+def workload_from_name(name):
+    """square (default, the headline layer), mlp_up, mlp_down, or
+    smallm_M_N_K (decode-like, e.g. smallm_16_12288_3072 = 16 rows, N=12288,
+    K=3072)."""
+    if name == "square":
+        return workloads.SQUARE
+    if name == "mlp_up":
+        return workloads.MLP_UP
+    if name == "mlp_down":
+        return workloads.MLP_DOWN
+    if name.startswith("smallm_"):
+        M, N, K = (int(v) for v in name.split("_")[1:4])
+        return workloads.Linear(f"small-m {M}x{K}->{N} g128", M=M, K=K, N=N, g=128, seed=3, bias=False)
+    raise SystemExit(f"unknown workload {name}")
+
+
+def n_sets_for(cfg):
+    """Enough independent operand sets that the ones a step touches total more
+    than 2x the 126 MB L2, so every step starts L2-cold (at least N_SETS)."""
+    per_set = 2 * cfg.M * cfg.K + cfg.N * cfg.K // 2 + 4 * (cfg.M + cfg.N) + 2 * cfg.M * cfg.N + cfg.M * cfg.K // 2
+    return max(N_SETS, -(-280_000_000 // per_set))
+
+
 def make_sets(cfg, w4, device):
-    """N_SETS independent (x, Wq, sw, bias, y) sets, resident in HBM."""
+    """Independent (x, Wq, sw, bias, y) sets, resident in HBM."""
     sets = []
     x0, W0, b0 = cfg.make()
-    for i in range(N_SETS):
+    for i in range(n_sets_for(cfg)):
         if i == 0:
             x, W, b = x0, W0, b0
         else:
             c = workloads.Linear(cfg.name, M=cfg.M, K=cfg.K, N=cfg.N, g=cfg.g, seed=cfg.seed + 100 * i,
-                                 outlier_frac=cfg.outlier_frac, outlier_scale=cfg.outlier_scale)
+                                 outlier_frac=cfg.outlier_frac, outlier_scale=cfg.outlier_scale, bias=cfg.bias,
+                                 act=cfg.act)
             x, W, b = c.make()
         xd = x.to(device)
         Wq, sw = w4.quantize_weight(W.to(device), cfg.g)
-        bd = b.to(device)
+        bd = b.to(device) if b is not None else None
         y = torch.empty(cfg.M, cfg.N, dtype=torch.bfloat16, device=device)
         Xq = torch.empty(cfg.M, cfg.K // 2, dtype=torch.int8, device=device)
         sx = torch.empty(cfg.M, dtype=torch.float32, device=device)
@@ -229,7 +259,7 @@ def run_impl(args, cfg, world, rank, local):
     g = cfg.g
 
     def fused(i):
-        s = sets[i % N_SETS]
+        s = sets[i % len(sets)]
         w4.linear_fused(s["x"], s["Wq"], s["sw"], s["b"], g, cfg.act, out=s["y"])
 
     # ---- the timed region: exactly `steps` fused layer calls
@@ -252,11 +282,11 @@ def run_impl(args, cfg, world, rank, local):
     # ---- per-kernel launch durations (same kernels and launch shapes, on the
     # launching stream) for the roofline of the dominant kernel
     def quant(i):
-        s = sets[i % N_SETS]
+        s = sets[i % len(sets)]
         w4.quantize_activation(s["x"], g, cfg.act, out=(s["Xq"], s["sx"]))
 
     def gemm(i):
-        s = sets[i % N_SETS]
+        s = sets[i % len(sets)]
         w4.linear(s["Xq"], s["sx"], s["Wq"], s["sw"], s["b"], out=s["y"])
 
     reps = max(args.steps, 20)
@@ -264,7 +294,7 @@ def run_impl(args, cfg, world, rank, local):
         quant(i)
         gemm(i)
     t_quant = time_loop(quant, reps, stream) / reps
-    for i in range(N_SETS):
+    for i in range(len(sets)):
         quant(i)
     t_gemm = time_loop(gemm, reps, stream) / reps
 
@@ -300,9 +330,21 @@ def run_impl(args, cfg, world, rank, local):
     hbm = peaks.get("hbm_gbs", FALLBACK["hbm_gbs"])
     quant_bytes = 2 * cfg.M * cfg.K + cfg.M * cfg.K // 2 + 4 * cfg.M
     roof_time = max(ops / (int8_peak * 1e12), cfg.bytes() / (hbm * 1e9))
+    small = cfg.M <= 64
+    if small:
+        # weight streaming: the packed weight dominates the bytes
+        k3_bytes = cfg.N * cfg.K // 2 + cfg.M * cfg.K // 2 + 4 * (cfg.M + cfg.N) + 2 * cfg.M * cfg.N
+        roof = {"bound": "hbm", "achieved": k3_bytes / t_gemm / 1e9, "peak": hbm, "unit": "GB/s",
+                "frac": k3_bytes / t_gemm / 1e9 / hbm, "traffic": MEASURED_TRAFFIC.get(("smallm", args.workload)),
+                "kernel": "smallm_kernel (split-K weight streaming)", "peak_note": f"{kind} HBM copy"}
+    else:
+        roof = {"bound": "tensor", "achieved": gemm_tops, "peak": int8_peak, "unit": "TOPS",
+                "frac": gemm_tops / int8_peak, "traffic": MEASURED_TRAFFIC.get(("gemm_tc", args.workload)),
+                "kernel": "gemm_tc_kernel (tcgen05 kind::i8, CTA pairs)",
+                "peak_note": f"int8 = 2 x {kind} bf16 burst {burst} TFLOP/s (nominal int8:bf16 ratio)"}
     cpu = None
     if world == 1 or rank == 0:
-        rows = 256
+        rows = min(256, cfg.M)
         t_cpu = time_oracle(cfg, rows)
         cpu = {"value": 2.0 * rows * cfg.N * cfg.K / t_cpu / 1e12, "unit": "TOPS", "cores": cpu_cores_used(),
                "kind": "oracle", "sample": f"{rows} of {cfg.M} rows, one pass, weights prepared offline"}
@@ -311,17 +353,15 @@ def run_impl(args, cfg, world, rank, local):
         "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "s4xs4->s32", "data": "synthetic",
-        "config": {"workload": cfg.name, "M": cfg.M, "K": cfg.K, "N": cfg.N, "g": cfg.g, "bias": True,
-                   "l2": f"{N_SETS} rotating input/weight/output sets (> 2x L2)",
+        "config": {"workload": cfg.name, "M": cfg.M, "K": cfg.K, "N": cfg.N, "g": cfg.g, "bias": cfg.bias,
+                   "gelu_input": bool(cfg.act),
+                   "l2": f"{len(sets)} rotating input/weight/output sets (> 2x L2)",
                    "parallelism": f"replicas x{world}"},
         "us_per_layer": ms_per_step * 1e3,
         "roofline_fraction_of_layer": roof_time / (ms_per_step / 1e3),
         "layer_roofline_us": roof_time * 1e6,
-        "kernels_us": {"rotate_quant_pack": t_quant * 1e6, "gemm_tc": t_gemm * 1e6},
-        "roofline": {"bound": "tensor", "achieved": gemm_tops, "peak": int8_peak, "unit": "TOPS",
-                     "frac": gemm_tops / int8_peak, "traffic": None,
-                     "kernel": "gemm_tc (tcgen05 kind::i8)",
-                     "peak_note": f"int8 = 2 x {kind} bf16 burst {burst} TFLOP/s"},
+        "kernels_us": {"rotate_quant_pack": t_quant * 1e6, ("smallm" if small else "gemm_tc"): t_gemm * 1e6},
+        "roofline": roof,
         "quant_kernel_roofline": {"bound": "hbm", "achieved": quant_bytes / t_quant / 1e9, "peak": hbm,
                                   "unit": "GB/s", "frac": quant_bytes / t_quant / 1e9 / hbm},
         "cpu_baseline": cpu,
@@ -336,14 +376,16 @@ def run_impl(args, cfg, world, rank, local):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--steps", type=int, default=4000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="square",
+                    help="square (default: 4608x3072->3072), mlp_up, mlp_down, or smallm_M_N_K")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     world, rank, local = dist_setup()
-    cfg = workloads.SQUARE
+    cfg = workload_from_name(args.workload)
     try:
         if args.impl == "reference":
             run_reference(args, cfg, world, rank)
