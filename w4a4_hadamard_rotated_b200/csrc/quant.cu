@@ -35,7 +35,10 @@
 //     the exact quotient only for values within ~4e-7 (relative) of a rounding
 //     boundary; exact ties with power-of-two scales stay exact.
 //   * Codes are stored low nibble first, 64 contiguous bytes per thread, with
-//     128-bit stores.
+//     128-bit stores.  A second output mode (used by the fused layer, whose
+//     tensor-core GEMM reads the activation operand as bytes) stores every
+//     code as one int8, 128 contiguous bytes per thread, from the same
+//     magic-number sums Horner-packed four per word.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -129,8 +132,15 @@ constexpr uint32_t kMagicBits = 0x4B400000u;   // bits of 1.5 * 2^23
 // Horner-packing eight sums (kMagicBits + n_e) as sum_e bits_e * 16^e leaves
 // this constant on top of the nibbles n_e (mod 2^32).
 constexpr uint32_t kHornerBias = kMagicBits * 0x11111111u;
+// The same for four sums per word in base 256 (one byte per code).
+constexpr uint32_t kHornerBias8 = kMagicBits * 0x01010101u;
+// Bytes n in 1..15 (code + 8) to the int8 codes n - 8, without borrows
+// between bytes: every byte is 0x81..0x8F before the subtraction.
+__device__ __forceinline__ uint32_t bytes_to_codes(uint32_t nb) {
+  return ((nb | 0x80808080u) - 0x08080808u) ^ 0x80808080u;
+}
 
-template <typename TIn, int G, int ACT>
+template <typename TIn, int G, int ACT, int OUT8>
 __global__ void __launch_bounds__(InTraits<TIn>::kMaxThreads, 1)
     rotate_quant_pack_kernel(const TIn* __restrict__ x, int64_t M, int K, int64_t ldx, int rows_per_tile,
                              int nstages, int8_t* __restrict__ out, float* __restrict__ scale,
@@ -276,6 +286,39 @@ __global__ void __launch_bounds__(InTraits<TIn>::kMaxThreads, 1)
     const float amax_r = __uint_as_float(row_amax[it % 3][p]);
     const float sc = amax_r / 7.0f;   // fp32 division, as the method states
     if (s == 0) scale[row] = sc;
+    if (OUT8) {
+      // one int8 code per byte: words w and w + 16 take elements 4w..4w+3 and
+      // 64+4w..64+4w+3 (the low and high halves of V[4w .. 4w+4))
+      uint32_t codes[kSlab / 4];
+      if (sc > 0.0f) {
+        const float ni = norm * (1.0f / sc);
+        const uint64_t magic2 = pk2(kMagic8, kMagic8);
+#pragma unroll
+        for (int w = 0; w < kHalf / 4; ++w) {
+          uint32_t lo_acc = 0u, hi_acc = 0u;
+#pragma unroll
+          for (int e = 3; e >= 0; --e) {
+            const int i = 4 * w + e;
+            const float m = (__popc((i / C) & L) & 1) ? -ni : ni;
+            const uint64_t f = add2(mul2(V[i], pk2(m, m)), magic2);
+            float f0, f1;
+            upk2(f, f0, f1);
+            lo_acc = lo_acc * 256u + __float_as_uint(f0);
+            hi_acc = hi_acc * 256u + __float_as_uint(f1);
+          }
+          codes[w] = bytes_to_codes(lo_acc - kHornerBias8);
+          codes[w + kHalf / 4] = bytes_to_codes(hi_acc - kHornerBias8);
+        }
+      } else {
+#pragma unroll
+        for (int w = 0; w < kSlab / 4; ++w) codes[w] = 0u;
+      }
+      uint4* dst = reinterpret_cast<uint4*>(out + row * static_cast<int64_t>(K) + static_cast<int64_t>(s) * kSlab);
+#pragma unroll
+      for (int w = 0; w < kSlab / 16; ++w)
+        dst[w] = make_uint4(codes[4 * w], codes[4 * w + 1], codes[4 * w + 2], codes[4 * w + 3]);
+      continue;
+    }
     uint32_t packed[kSlab / 8];
     if (sc > 0.0f) {
       const float ni = norm * (1.0f / sc);
@@ -329,7 +372,7 @@ static void rq_shape(int S, int max_threads, int* P, int* threads) {
   *threads = ((p * S + 31) / 32) * 32;
 }
 
-template <typename TIn, int G, int ACT>
+template <typename TIn, int G, int ACT, int OUT8>
 static cudaError_t launch_rq(const TIn* x, int64_t M, int K, int64_t ldx, int8_t* out, float* scale, int num_sms,
                              unsigned int* status, cudaStream_t stream) {
   const int S = K / kSlab;
@@ -341,7 +384,7 @@ static cudaError_t launch_rq(const TIn* x, int64_t M, int K, int64_t ldx, int8_t
   if (nst > kMaxStages) nst = kMaxStages;
   if (nst < 1) return cudaErrorInvalidValue;
   const size_t smem = nst * stage_bytes;
-  auto kern = rotate_quant_pack_kernel<TIn, G, ACT>;
+  auto kern = rotate_quant_pack_kernel<TIn, G, ACT, OUT8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const int64_t tiles = (M + P - 1) / P;
@@ -350,29 +393,34 @@ static cudaError_t launch_rq(const TIn* x, int64_t M, int K, int64_t ldx, int8_t
   return cudaGetLastError();
 }
 
-template <typename TIn>
+template <typename TIn, int OUT8>
 static cudaError_t dispatch_rq(const TIn* x, int64_t M, int K, int64_t ldx, int g, int act, int8_t* out,
                                float* scale, int num_sms, unsigned int* status, cudaStream_t stream) {
   if (act == 0) {
-    if (g == 64) return launch_rq<TIn, 64, 0>(x, M, K, ldx, out, scale, num_sms, status, stream);
-    if (g == 128) return launch_rq<TIn, 128, 0>(x, M, K, ldx, out, scale, num_sms, status, stream);
-    if (g == 256) return launch_rq<TIn, 256, 0>(x, M, K, ldx, out, scale, num_sms, status, stream);
+    if (g == 64) return launch_rq<TIn, 64, 0, OUT8>(x, M, K, ldx, out, scale, num_sms, status, stream);
+    if (g == 128) return launch_rq<TIn, 128, 0, OUT8>(x, M, K, ldx, out, scale, num_sms, status, stream);
+    if (g == 256) return launch_rq<TIn, 256, 0, OUT8>(x, M, K, ldx, out, scale, num_sms, status, stream);
   } else {
-    if (g == 64) return launch_rq<TIn, 64, 1>(x, M, K, ldx, out, scale, num_sms, status, stream);
-    if (g == 128) return launch_rq<TIn, 128, 1>(x, M, K, ldx, out, scale, num_sms, status, stream);
-    if (g == 256) return launch_rq<TIn, 256, 1>(x, M, K, ldx, out, scale, num_sms, status, stream);
+    if (g == 64) return launch_rq<TIn, 64, 1, OUT8>(x, M, K, ldx, out, scale, num_sms, status, stream);
+    if (g == 128) return launch_rq<TIn, 128, 1, OUT8>(x, M, K, ldx, out, scale, num_sms, status, stream);
+    if (g == 256) return launch_rq<TIn, 256, 1, OUT8>(x, M, K, ldx, out, scale, num_sms, status, stream);
   }
   return cudaErrorInvalidValue;
 }
 
 cudaError_t rotate_quant_bf16(const uint16_t* x, int64_t M, int K, int64_t ldx, int g, int act, int8_t* out,
                               float* scale, int num_sms, unsigned int* status, cudaStream_t stream) {
-  return dispatch_rq<uint16_t>(x, M, K, ldx, g, act, out, scale, num_sms, status, stream);
+  return dispatch_rq<uint16_t, 0>(x, M, K, ldx, g, act, out, scale, num_sms, status, stream);
+}
+
+cudaError_t rotate_quant_bf16_i8(const uint16_t* x, int64_t M, int K, int64_t ldx, int g, int act, int8_t* out,
+                                 float* scale, int num_sms, unsigned int* status, cudaStream_t stream) {
+  return dispatch_rq<uint16_t, 1>(x, M, K, ldx, g, act, out, scale, num_sms, status, stream);
 }
 
 cudaError_t rotate_quant_f32(const float* x, int64_t M, int K, int64_t ldx, int g, int8_t* out, float* scale,
                              int num_sms, unsigned int* status, cudaStream_t stream) {
-  return dispatch_rq<float>(x, M, K, ldx, g, 0, out, scale, num_sms, status, stream);
+  return dispatch_rq<float, 0>(x, M, K, ldx, g, 0, out, scale, num_sms, status, stream);
 }
 
 }  // namespace w4a4
