@@ -211,7 +211,7 @@ def workload_from_name(name):
 def n_sets_for(cfg):
     """Enough independent operand sets that the ones a step touches total more
     than 2x the 126 MB L2, so every step starts L2-cold (at least N_SETS)."""
-    per_set = 2 * cfg.M * cfg.K + cfg.N * cfg.K // 2 + 4 * (cfg.M + cfg.N) + 2 * cfg.M * cfg.N + cfg.M * cfg.K
+    per_set = 2 * cfg.M * cfg.K + cfg.N * cfg.K // 2 + 4 * (cfg.M + cfg.N) + 2 * cfg.M * cfg.N + cfg.M * cfg.K // 2
     return max(N_SETS, -(-280_000_000 // per_set))
 
 
@@ -232,9 +232,8 @@ def make_sets(cfg, w4, device):
         bd = b.to(device) if b is not None else None
         y = torch.empty(cfg.M, cfg.N, dtype=torch.bfloat16, device=device)
         Xq = torch.empty(cfg.M, cfg.K // 2, dtype=torch.int8, device=device)
-        Xc = torch.empty(cfg.M, cfg.K, dtype=torch.int8, device=device) if cfg.M > 64 else None
         sx = torch.empty(cfg.M, dtype=torch.float32, device=device)
-        sets.append({"x": xd, "Wq": Wq, "sw": sw, "b": bd, "y": y, "Xq": Xq, "Xc": Xc, "sx": sx})
+        sets.append({"x": xd, "Wq": Wq, "sw": sw, "b": bd, "y": y, "Xq": Xq, "sx": sx})
     torch.cuda.synchronize()
     return sets
 
@@ -286,22 +285,12 @@ def run_impl(args, cfg, world, rank, local):
 
     def quant(i):
         s = sets[i % len(sets)]
-        if small:
-            w4.quantize_activation(s["x"], g, cfg.act, out=(s["Xq"], s["sx"]))
-        else:
-            w4.quantize_activation_i8(s["x"], g, cfg.act, out=(s["Xc"], s["sx"]))
+        w4.quantize_activation(s["x"], g, cfg.act, out=(s["Xq"], s["sx"]))
 
     def gemm(i):
         s = sets[i % len(sets)]
-        if small:
-            w4.linear(s["Xq"], s["sx"], s["Wq"], s["sw"], s["b"], out=s["y"])
-        else:
-            w4.linear_i8(s["Xc"], s["sx"], s["Wq"], s["sw"], s["b"], out=s["y"])
-
-    def gemm_packed(i):
-        # the packed-activation tensor-core kernel of w4a4_linear, for reference
-        s = sets[i % len(sets)]
         w4.linear(s["Xq"], s["sx"], s["Wq"], s["sw"], s["b"], out=s["y"])
+
 
     reps = max(min(args.steps, 2000), 20)
     for i in range(3):
@@ -311,12 +300,6 @@ def run_impl(args, cfg, world, rank, local):
     for i in range(len(sets)):
         quant(i)
     t_gemm = time_loop(gemm, reps, stream) / reps
-    t_gemm_packed = None
-    if not small:
-        for i in range(len(sets)):
-            w4.quantize_activation(sets[i]["x"], g, cfg.act, out=(sets[i]["Xq"], sets[i]["sx"]))
-        gemm_packed(0)
-        t_gemm_packed = time_loop(gemm_packed, reps, stream) / reps
 
     # ---- end to end through the public API with host buffers: pinned x in,
     # y out, copies inside the timed region
@@ -348,7 +331,7 @@ def run_impl(args, cfg, world, rank, local):
     int8_peak = burst * INT8_OVER_BF16
     gemm_tops = ops / t_gemm / 1e12
     hbm = peaks.get("hbm_gbs", FALLBACK["hbm_gbs"])
-    quant_bytes = 2 * cfg.M * cfg.K + (cfg.M * cfg.K // 2 if small else cfg.M * cfg.K) + 4 * cfg.M
+    quant_bytes = 2 * cfg.M * cfg.K + cfg.M * cfg.K // 2 + 4 * cfg.M
     roof_time = max(ops / (int8_peak * 1e12), cfg.bytes() / (hbm * 1e9))
     if small:
         # weight streaming: the packed weight dominates the bytes
@@ -358,8 +341,8 @@ def run_impl(args, cfg, world, rank, local):
                 "kernel": "smallm_kernel (split-K weight streaming)", "peak_note": f"{kind} HBM copy"}
     else:
         roof = {"bound": "tensor", "achieved": gemm_tops, "peak": int8_peak, "unit": "TOPS",
-                "frac": gemm_tops / int8_peak, "traffic": MEASURED_TRAFFIC.get(("gemm_ts", args.workload)),
-                "kernel": "gemm_ts_kernel (tcgen05 kind::i8, weights widened into tensor memory, CTA pairs)",
+                "frac": gemm_tops / int8_peak, "traffic": MEASURED_TRAFFIC.get(("gemm_tc", args.workload)),
+                "kernel": "gemm_tc_kernel (tcgen05 kind::i8, packed operands widened in shared memory, CTA pairs)",
                 "peak_note": f"int8 = 2 x {kind} bf16 burst {burst} TFLOP/s (nominal int8:bf16 ratio)"}
     cpu = None
     if world == 1 or rank == 0:
@@ -379,9 +362,7 @@ def run_impl(args, cfg, world, rank, local):
         "us_per_layer": ms_per_step * 1e3,
         "roofline_fraction_of_layer": roof_time / (ms_per_step / 1e3),
         "layer_roofline_us": roof_time * 1e6,
-        "kernels_us": {("rotate_quant_pack" if small else "rotate_quant_i8"): t_quant * 1e6,
-                       ("smallm" if small else "gemm_ts"): t_gemm * 1e6,
-                       **({} if small else {"gemm_tc_packed_operands": t_gemm_packed * 1e6})},
+        "kernels_us": {"rotate_quant_pack": t_quant * 1e6, ("smallm" if small else "gemm_tc"): t_gemm * 1e6},
         "roofline": roof,
         "quant_kernel_roofline": {"bound": "hbm", "achieved": quant_bytes / t_quant / 1e9, "peak": hbm,
                                   "unit": "GB/s", "frac": quant_bytes / t_quant / 1e9 / hbm},

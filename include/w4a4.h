@@ -106,11 +106,8 @@ int w4a4_linear(const int8_t* Xq, const float* sx, const int8_t* Wq, const float
                 int64_t ldy, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
- * Fused layer: rotate + quantise the activation, then the W4A4 linear, with
- * the quantised activation and its scales kept in the workspace.  M <= 64:
- * w4a4_quantize_activation + the weight-streaming kernel of w4a4_linear;
- * larger M: w4a4_quantize_activation_i8 + w4a4_linear_i8.  Same result
- * either way (the codes and the int32 accumulators are the same).
+ * Fused layer: w4a4_quantize_activation followed by w4a4_linear, with the
+ * packed activation and its scales kept in the workspace.
  *   x [M, K] bf16 bits with row stride ldx; other arguments as above.
  *   workspace: at least w4a4_fused_workspace_bytes(M, N, K) bytes, laid out as
  *       [small-M scratch, counter block first][quantised x][sx]; the same rule
@@ -121,48 +118,6 @@ int w4a4_linear_fused(const uint16_t* x, int64_t ldx, const int8_t* Wq, const fl
                       const uint16_t* bias, uint16_t* y, int64_t ldy, int64_t M, int64_t N,
                       int64_t K, int g, int act, void* workspace, size_t workspace_bytes,
                       void* stream);
-
-/*
- * Activation preparation for the tensor-core GEMM: the same rotation and
- * quantisation as w4a4_quantize_activation (same codes, same scales), but
- * every code is stored as one int8 (the value q in [-7, 7]) instead of two
- * per byte.  The pages pack two codes per byte because their GEMM consumes
- * nibbles; tcgen05 has no 4-bit integer kind, so the sm_100a GEMM reads
- * bytes, and the fused layer hands it this form so that the activation tile
- * goes from HBM to the tensor cores without a widening pass.
- *   x   [M, K] bf16 bits, row stride ldx >= K, 16-byte aligned, ldx % 8 == 0
- *   act 0: none; 1: exact-erf GELU applied to x before the rotation
- *   Xc  [M, K] int8 output (contiguous rows, 16-byte aligned); sx [M] fp32
- *   M >= 0 (M == 0 is a no-op); K % 128 == 0, K % g == 0, 128 <= K <= 32768.
- */
-int w4a4_quantize_activation_i8(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int g,
-                                int act, int8_t* Xc, float* sx, void* stream);
-
-/*
- * W4A4 linear on activation codes stored one per byte (from
- * w4a4_quantize_activation_i8) and packed weights (from
- * w4a4_quantize_weight): the s4 x s4 GEMM with int32 accumulation and the
- * rank-one epilogue of the page's Description, on the tcgen05 tensor cores
- * (packed weights widened into tensor memory, 256 x 192 tiles on CTA pairs).
- *   Xc [M, K] int8 codes in [-7, 7], contiguous rows, 16-byte aligned; sx [M] fp32
- *   Wq [N, K/2] packed int4, sw [N] fp32; bias [N] bf16 bits or NULL
- *   y  [M, N] bf16 bits output, row stride ldy >= N, ldy % 8 == 0, 16-byte aligned
- *   M >= 0, N >= 1, N % 8 == 0, 32 <= K <= 131072, K % 32 == 0.
- * No workspace.  The int32 accumulators equal those of w4a4_linear on the
- * same codes, so the output is bit-identical to it.
- */
-int w4a4_linear_i8(const int8_t* Xc, const float* sx, const int8_t* Wq, const float* sw,
-                   const uint16_t* bias, uint16_t* y, int64_t M, int64_t N, int64_t K, int64_t ldy,
-                   void* stream);
-
-/*
- * Raw int32 accumulators acc[m, n] = sum_k Xc[m, k] * qw[n, k] of the
- * w4a4_linear_i8 kernel (no epilogue), for bit-exact checks.
- *   acc [M, N] int32 output with row stride ldc >= N, ldc % 4 == 0.
- * Other rules as for w4a4_linear_i8.
- */
-int w4a4_gemm_s32_i8(const int8_t* Xc, const int8_t* Wq, int32_t* acc, int64_t M, int64_t N,
-                     int64_t K, int64_t ldc, void* stream);
 
 /* Workspace sizes in bytes (0 when none is needed).  Pure host functions. */
 size_t w4a4_workspace_bytes(int64_t M, int64_t N, int64_t K);

@@ -13,9 +13,6 @@ Functions keep the C names without the ``w4a4_`` prefix:
   linear(Xq, sx, Wq, sw, bias=None)          -> y [M, N] bf16
   linear_fused(x, Wq, sw, bias=None, g, act) -> y [M, N] bf16
   gemm_s32(Xq, Wq, path=0)                   -> acc [M, N] int32
-  quantize_activation_i8(x, g, act=0)        -> (Xc [M, K] int8, sx [M] fp32)
-  linear_i8(Xc, sx, Wq, sw, bias=None)       -> y [M, N] bf16
-  gemm_s32_i8(Xc, Wq)                        -> acc [M, N] int32
 """
 
 import ctypes
@@ -47,9 +44,7 @@ SIGNATURES = {
     "w4a4_fused_workspace_bytes": (_SZ, [_I64, _I64, _I64]),
     "w4a4_gemm_s32": (_I, [_P, _P, _P, _I64, _I64, _I64, _I64, _I, _P, _SZ, _P]),
     "w4a4_linear_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P]),
-    "w4a4_quantize_activation_i8": (_I, [_P, _I64, _I64, _I64, _I, _I, _P, _P, _P]),
-    "w4a4_linear_i8": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P]),
-    "w4a4_gemm_s32_i8": (_I, [_P, _P, _P, _I64, _I64, _I64, _I64, _P]),
+
     "w4a4_last_device_error": (_I, [_P]),
     "w4a4_debug_wait_timeout": (_I, [_I64, _P]),
 }
@@ -199,51 +194,6 @@ def gemm_s32(Xq, Wq, path=0, out=None):
     ws = workspace(nbytes, Xq.device) if nbytes else None
     _check(lib.w4a4_gemm_s32(_ptr(Xq), _ptr(Wq), _ptr(acc), M, N, K, acc.stride(0), path, _ptr(ws), nbytes,
                              _stream(Xq)), "w4a4_gemm_s32")
-    return acc
-
-
-def quantize_activation_i8(x, g=128, act=0, out=None):
-    """Rotate + quantise bf16 activations x [M, K] -> (Xc [M, K] int8 codes, one
-    per byte, sx [M] fp32): the operand form of the tensor-core GEMM."""
-    lib = load_library()
-    _need_cuda(x, torch.bfloat16, "x")
-    if x.dim() != 2 or x.stride(1) != 1:
-        raise ValueError("x must be a 2-D tensor with a contiguous inner dimension")
-    M, K = x.shape
-    if out is None:
-        Xc = torch.empty(M, K, dtype=torch.int8, device=x.device)
-        sx = torch.empty(M, dtype=torch.float32, device=x.device)
-    else:
-        Xc, sx = out
-    _check(lib.w4a4_quantize_activation_i8(_ptr(x), M, K, x.stride(0), g, act, _ptr(Xc), _ptr(sx), _stream(x)),
-           "w4a4_quantize_activation_i8")
-    return Xc, sx
-
-
-def linear_i8(Xc, sx, Wq, sw, bias=None, out=None):
-    """y [M, N] bf16 from activation codes one per byte (Xc [M, K] int8) and
-    packed weights."""
-    lib = load_library()
-    _need_cuda(Xc, torch.int8, "Xc")
-    _need_cuda(Wq, torch.int8, "Wq")
-    M, K = Xc.shape
-    N = Wq.shape[0]
-    y = out if out is not None else torch.empty(M, N, dtype=torch.bfloat16, device=Xc.device)
-    _check(lib.w4a4_linear_i8(_ptr(Xc), _ptr(sx), _ptr(Wq), _ptr(sw), _ptr(bias), _ptr(y), M, N, K, y.stride(0),
-                              _stream(Xc)), "w4a4_linear_i8")
-    return y
-
-
-def gemm_s32_i8(Xc, Wq, out=None):
-    """Raw int32 accumulators acc [M, N] of the linear_i8 kernel."""
-    lib = load_library()
-    _need_cuda(Xc, torch.int8, "Xc")
-    _need_cuda(Wq, torch.int8, "Wq")
-    M, K = Xc.shape
-    N = Wq.shape[0]
-    acc = out if out is not None else torch.empty(M, N, dtype=torch.int32, device=Xc.device)
-    _check(lib.w4a4_gemm_s32_i8(_ptr(Xc), _ptr(Wq), _ptr(acc), M, N, K, acc.stride(0), _stream(Xc)),
-           "w4a4_gemm_s32_i8")
     return acc
 
 

@@ -91,38 +91,6 @@ int packed_map(CUtensorMap* map, const int8_t* base, int64_t rows, int64_t K, in
 
 namespace {
 
-// 2-D map over a byte matrix [rows, cols] with row stride ld bytes (a multiple
-// of 16), box {box_cols, box_rows}; out-of-range elements read as zero.
-int byte_map(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int64_t ld, int box_cols, int box_rows,
-             CUtensorMapSwizzle swizzle) {
-  EncodeTiledFn fn = encode_fn();
-  if (fn == nullptr) return W4A4_ERR_CUDA;
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld)};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
-  const cuuint32_t estr[2] = {1u, 1u};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? W4A4_OK : W4A4_ERR_CUDA;
-}
-
-// 2-D map over a bf16 output [rows, cols] with row stride ld (elements), box
-// {32, 32}, no swizzle (the staging layout of the weights-in-tensor-memory
-// GEMM's epilogue).
-int output_map_plain(CUtensorMap* map, void* base, int64_t rows, int64_t cols, int64_t ld) {
-  EncodeTiledFn fn = encode_fn();
-  if (fn == nullptr) return W4A4_ERR_CUDA;
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld * 2)};
-  const cuuint32_t box[2] = {32u, 32u};
-  const cuuint32_t estr[2] = {1u, 1u};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? W4A4_OK : W4A4_ERR_CUDA;
-}
-
 // 2-D map over a bf16 output [rows, cols] with row stride ld (elements), box
 // {32, 32}, 64-byte swizzle (the epilogue's staging layout).
 int output_map(CUtensorMap* map, void* base, int64_t rows, int64_t cols, int64_t ld) {
@@ -171,7 +139,8 @@ int check_gemm_shape(int64_t M, int64_t N, int64_t K) {
 }
 
 
-// Shared body of w4a4_linear / w4a4_gemm_s32 after validation.
+// Shared body of w4a4_linear / w4a4_gemm_s32 after validation.  path 0: the
+// tcgen05 tensor-core kernel; 1: the small-M weight-streaming kernel.
 int run_linear(const int8_t* Xq, const float* sx, const int8_t* Wq, const float* sw, const uint16_t* bias, void* out,
                int64_t M, int64_t N, int64_t K, int64_t ldo, int out_s32, int path, void* ws, size_t ws_bytes,
                cudaStream_t stream) {
@@ -223,35 +192,6 @@ int run_linear(const int8_t* Xq, const float* sx, const int8_t* Wq, const float*
   a.out_s32 = out_s32;
   a.status = dev->status;
   return gemm_tc_launch(tmA, tmB, tmY, a, dev->num_sms, stream) == cudaSuccess ? W4A4_OK : W4A4_ERR_CUDA;
-}
-
-// The weights-in-tensor-memory GEMM on activation codes stored one per byte.
-int run_linear_ts(const int8_t* Xc, const float* sx, const int8_t* Wq, const float* sw, const uint16_t* bias,
-                  void* out, int64_t M, int64_t N, int64_t K, int64_t ldo, int out_s32, cudaStream_t stream) {
-  DeviceInfo* dev = nullptr;
-  int st = current_device(&dev);
-  if (st != W4A4_OK) return st;
-  if (M == 0) return W4A4_OK;
-  CUtensorMap tmAct, tmW, tmY;
-  if ((st = byte_map(&tmAct, Xc, M, K, K, 128, kTsTileA / 2, CU_TENSOR_MAP_SWIZZLE_128B)) != W4A4_OK) return st;
-  if ((st = byte_map(&tmW, Wq, N, K / 2, K / 2, 64, kTsTileW / 2, CU_TENSOR_MAP_SWIZZLE_64B)) != W4A4_OK) return st;
-  if (out_s32) {
-    tmY = tmAct;   // not read by the int32 epilogue
-  } else if ((st = output_map_plain(&tmY, out, M, N, ldo)) != W4A4_OK) {
-    return st;
-  }
-  GemmArgs a{};
-  a.M = M;
-  a.N = N;
-  a.K = K;
-  a.sx = sx;
-  a.sw = sw;
-  a.bias = bias;
-  a.out = out;
-  a.ldo = ldo;
-  a.out_s32 = out_s32;
-  a.status = dev->status;
-  return gemm_ts_launch(tmAct, tmW, tmY, a, dev->num_sms, stream) == cudaSuccess ? W4A4_OK : W4A4_ERR_CUDA;
 }
 
 __global__ void wait_forever_bounded_kernel(unsigned long long limit_ns, unsigned int* status) {
@@ -347,38 +287,6 @@ int w4a4_quantize_activation(const uint16_t* x, int64_t M, int64_t K, int64_t ld
              : W4A4_ERR_CUDA;
 }
 
-int w4a4_quantize_activation_i8(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int g, int act, int8_t* Xc,
-                                float* sx, void* stream) {
-  if (M != 0 && (x == nullptr || Xc == nullptr || sx == nullptr)) return W4A4_ERR_NULL;
-  int st = check_quant_shape(K, g);
-  if (st != W4A4_OK) return st;
-  if (act != 0 && act != 1) return W4A4_ERR_ARG;
-  if (M < 0 || M > (int64_t(1) << 26)) return W4A4_ERR_SHAPE;
-  if (ldx < K) return W4A4_ERR_SHAPE;
-  if (ldx % 8 != 0 || !aligned(x, 16) || !aligned(Xc, 16) || !aligned(sx, 4)) return W4A4_ERR_ALIGN;
-  DeviceInfo* dev = nullptr;
-  if ((st = current_device(&dev)) != W4A4_OK) return st;
-  if (M == 0) return W4A4_OK;
-  return rotate_quant_bf16_i8(x, M, static_cast<int>(K), ldx, g, act, Xc, sx, dev->num_sms, dev->status,
-                              static_cast<cudaStream_t>(stream)) == cudaSuccess
-             ? W4A4_OK
-             : W4A4_ERR_CUDA;
-}
-
-int w4a4_linear_i8(const int8_t* Xc, const float* sx, const int8_t* Wq, const float* sw, const uint16_t* bias,
-                   uint16_t* y, int64_t M, int64_t N, int64_t K, int64_t ldy, void* stream) {
-  int st = validate_linear(Xc, sx, Wq, sw, bias, y, M, N, K, ldy, 0);
-  if (st != W4A4_OK) return st;
-  return run_linear_ts(Xc, sx, Wq, sw, bias, y, M, N, K, ldy, 0, static_cast<cudaStream_t>(stream));
-}
-
-int w4a4_gemm_s32_i8(const int8_t* Xc, const int8_t* Wq, int32_t* acc, int64_t M, int64_t N, int64_t K, int64_t ldc,
-                     void* stream) {
-  int st = validate_linear(Xc, nullptr, Wq, nullptr, nullptr, acc, M, N, K, ldc, 1);
-  if (st != W4A4_OK) return st;
-  return run_linear_ts(Xc, nullptr, Wq, nullptr, nullptr, acc, M, N, K, ldc, 1, static_cast<cudaStream_t>(stream));
-}
-
 size_t w4a4_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   if (M <= 0 || N <= 0 || K <= 0) return 0;
   if (M <= smallm_threshold()) return smallm_workspace_bytes(M, N, K);
@@ -393,11 +301,9 @@ static size_t fused_linear_part(int64_t M, int64_t N, int64_t K) {
   return round256(lin > kSmallMCounterBytes ? lin : kSmallMCounterBytes);
 }
 
-// Bytes of the quantised activation in the fused workspace: packed codes for
-// the small-M kernel, one int8 per code for the tensor-core kernel.
+// Bytes of the packed activation in the fused workspace.
 static size_t fused_codes_bytes(int64_t M, int64_t K) {
-  const size_t per_row = M <= smallm_threshold() ? static_cast<size_t>(K / 2) : static_cast<size_t>(K);
-  return round256(static_cast<size_t>(M) * per_row);
+  return round256(static_cast<size_t>(M) * static_cast<size_t>(K / 2));
 }
 
 size_t w4a4_fused_workspace_bytes(int64_t M, int64_t N, int64_t K) {
@@ -452,14 +358,9 @@ int w4a4_linear_fused(const uint16_t* x, int64_t ldx, const int8_t* Wq, const fl
   int8_t* xq = reinterpret_cast<int8_t*>(ws + lin_bytes);
   float* sx = reinterpret_cast<float*>(ws + lin_bytes + fused_codes_bytes(M, K));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (M <= smallm_threshold()) {
-    // packed codes into the weight-streaming kernel
-    if ((st = w4a4_quantize_activation(x, M, K, ldx, g, act, xq, sx, stream)) != W4A4_OK) return st;
-    return run_linear(xq, sx, Wq, sw, bias, y, M, N, K, ldy, 0, 1, ws, lin_bytes, s);
-  }
-  // one int8 per code into the tensor-core kernel
-  if ((st = w4a4_quantize_activation_i8(x, M, K, ldx, g, act, xq, sx, stream)) != W4A4_OK) return st;
-  return run_linear_ts(xq, sx, Wq, sw, bias, y, M, N, K, ldy, 0, s);
+  if ((st = w4a4_quantize_activation(x, M, K, ldx, g, act, xq, sx, stream)) != W4A4_OK) return st;
+  const int path = (M <= smallm_threshold()) ? 1 : 0;
+  return run_linear(xq, sx, Wq, sw, bias, y, M, N, K, ldy, 0, path, ws, lin_bytes, s);
 }
 
 int w4a4_last_device_error(void* stream) {

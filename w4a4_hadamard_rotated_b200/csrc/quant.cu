@@ -5,40 +5,42 @@
 //
 // B200 design (an HBM-bound pass that is close to ALU-bound as well: 2 bytes
 // read, half a byte written, ~log2(g) adds per code)
-//   * Every row is split into S = K/128 slabs of 128 consecutive elements and
-//     each thread owns one slab, entirely in registers, as 64 packed fp32
-//     pairs (element i, element i + 64).  Six radix-2 Walsh-Hadamard stages run
-//     as paired sm_100 add/sub.f32x2 instructions (two lanes per instruction),
-//     the seventh (distance 64, g >= 128) pairs the two halves of a register;
-//     g = 256 spans two slabs held by adjacent lanes and takes one shuffle
-//     stage.
+//   * Every row is split into S = K/64 slabs of 64 consecutive elements and
+//     each thread owns one slab in registers, as 32 packed fp32 pairs
+//     (element i, element i + 32).  Five radix-2 Walsh-Hadamard stages run as
+//     paired sm_100 add/sub.f32x2 instructions, the sixth (distance 32) pairs
+//     the two halves of a register; g = 128 and g = 256 span two and four
+//     slabs held by neighbouring lanes and take one and two shuffle stages.
+//     At about 100 registers per thread, two or three CTAs share an SM, so the
+//     latency of one CTA's barrier and loads hides behind the others' math.
 //   * The kernel is persistent: a CTA walks row tiles (P whole rows) with a
 //     grid stride, and one thread streams the rows of the coming tiles into a
-//     3-4 deep shared-memory ring with bulk-async (TMA) copies, so HBM reads
-//     stay in flight during the arithmetic and every SM gets the same, fully
-//     coalesced request pattern.  The one CTA barrier per tile (for the row
-//     amax) also frees the ring slot that tile used.
+//     shared-memory ring with bulk-async (TMA) copies, so HBM reads stay in
+//     flight during the arithmetic.  P is chosen on the host so that the rows
+//     spread evenly over the resident CTAs.  The one CTA barrier per tile (for
+//     the row amax) also frees the ring slot that tile used.
 //   * A lane reads its slab from shared memory in XOR-swizzled 16-byte chunks
 //     (chunk j from position j ^ L, L = lane & 7), which keeps the 128-bit
-//     shared loads free of bank conflicts.  Permuting the input of a Walsh-Hadamard
-//     transform by an XOR of the index only flips signs of the output:
-//     H(x[. ^ a])[i] = (-1)^popcount(i & a) H(x)[i].  The sign of each output
-//     chunk is folded into the quantisation multiplier; the quantiser is odd
-//     (round-half-even and the clamp are symmetric), so the codes are exact.
+//     shared loads free of bank conflicts.  Permuting the input of a
+//     Walsh-Hadamard transform by an XOR of the index only flips signs of the
+//     output: H(x[. ^ a])[i] = (-1)^popcount(i & a) H(x)[i].  The shuffle
+//     stages combine lanes whose swizzles differ in one bit, which makes the
+//     partner's value a known sign times the true one; the remaining sign of
+//     each output chunk is folded into the quantisation multiplier, and the
+//     quantiser is odd (round-half-even and the clamp are symmetric), so the
+//     codes are exact.
 //   * The row amax is reduced with shared-memory atomics on the float bits
 //     (triple-buffered slots, one barrier per tile), and s = amax / 7 in fp32.
-//     The code is round-half-even of r * (1/s) in fp32: a reciprocal multiply
-//     (with 1/sqrt(g) and the chunk sign folded in) and a magic-number rounding
-//     put the code in the low mantissa bits, and a Horner chain of integer
-//     multiply-adds packs 8 codes per word as they are made.  The product is
-//     within 3 ulp of the quotient r / s, so a code can differ from the one of
-//     the exact quotient only for values within ~4e-7 (relative) of a rounding
-//     boundary; exact ties with power-of-two scales stay exact.
-//   * Codes are stored low nibble first, 64 contiguous bytes per thread, with
-//     128-bit stores.  A second output mode (used by the fused layer, whose
-//     tensor-core GEMM reads the activation operand as bytes) stores every
-//     code as one int8, 128 contiguous bytes per thread, from the same
-//     magic-number sums Horner-packed four per word.
+//     The code is round-half-even of u * (norm/s): one fused multiply-add of
+//     the butterfly sum u by the reciprocal multiplier (with 1/sqrt(g) and the
+//     chunk sign folded in) and a magic number rounds the exact product to an
+//     integer and leaves it in the low mantissa bits, and a Horner chain of
+//     integer multiply-adds packs 8 codes per word as they are made.  The
+//     multiplier is within 2 ulp of 1/s, so a code can differ from the one of
+//     the exact quotient r / s only for values within ~3e-7 (relative) of a
+//     rounding boundary; exact ties with power-of-two scales stay exact.
+//   * Codes are stored low nibble first, 32 contiguous bytes per thread, with
+//     128-bit stores.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -49,24 +51,24 @@
 
 namespace w4a4 {
 
-constexpr int kSlab = 128;     // elements per thread
-constexpr int kHalf = 64;      // packed pairs per thread
+constexpr int kSlab = 64;      // elements per thread
+constexpr int kHalf = 32;      // packed pairs per thread
 constexpr int kMaxRows = 64;   // rows per CTA tile
+constexpr int kMaxThreads = 512;
+constexpr int kMaxStages = 4;
+constexpr int kMinStages = 2;
+constexpr size_t kRingBytesPerSm = 200 * 1024;   // shared memory for the rings of one SM
 
 template <typename TIn>
 struct InTraits;
 template <>
 struct InTraits<uint16_t> {  // bf16 bits
   static constexpr int kChunkElems = 8;
-  static constexpr int kMaxThreads = 256;
 };
 template <>
 struct InTraits<float> {     // fp32 weights (offline)
   static constexpr int kChunkElems = 4;
-  static constexpr int kMaxThreads = 192;
 };
-constexpr int kMaxStages = 4;
-constexpr size_t kRingBytes = 200 * 1024;   // shared memory for the row ring
 
 // ---- packed fp32 pairs (sm_100 .f32x2 arithmetic)
 __device__ __forceinline__ uint64_t pk2(float a, float b) {
@@ -87,16 +89,6 @@ __device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
   asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
   return r;
 }
-__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t r;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-  return r;
-}
 
 __device__ __forceinline__ float gelu_erf(float t) {
   return 0.5f * t * (1.0f + erff(t * 0.70710678118654752f));
@@ -111,7 +103,7 @@ __device__ __forceinline__ float elem(const uint4 w, int e, const float*) {
   return __uint_as_float(e == 0 ? w.x : (e == 1 ? w.y : (e == 2 ? w.z : w.w)));
 }
 
-// One radix-2 butterfly stage at distance H (< 64) over the packed pairs.
+// One radix-2 butterfly stage at distance H (< 32) over the packed pairs.
 template <int H>
 __device__ __forceinline__ void fht_stage2(uint64_t (&V)[kHalf]) {
 #pragma unroll
@@ -125,6 +117,33 @@ __device__ __forceinline__ void fht_stage2(uint64_t (&V)[kHalf]) {
   }
 }
 
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+
+// Butterfly stage across lanes: the group's two halves at distance 64 * D
+// (D = 1 or 2) are held by lanes l and l ^ D.  Values are kept "twisted":
+// V[i] holds t(i) times the true value, with a sign t(i) that depends only on
+// the lane and i.  The partner's swizzle differs in bit log2(D), so its twist
+// differs from ours by rho(i) = (-1)^bit(log2 D) of the chunk index -- the
+// same for both halves of V[i], which lie 4 chunks (bf16) or 8 chunks (fp32)
+// apart.  With sigma = +1 in the lower half and -1 in the upper half, the
+// new twisted value is sigma * own + rho * partner; this stage stores rho
+// times it, fma(own, sigma * rho, partner), and the extra factor rho(i) joins
+// the twist that the quantiser multiplier undoes.
+template <int D, int C>
+__device__ __forceinline__ void fht_cross(uint64_t (&V)[kHalf], bool upper) {
+  const float sg = upper ? -1.0f : 1.0f;
+  const uint64_t sr_pos = pk2(sg, sg), sr_neg = pk2(-sg, -sg);
+#pragma unroll
+  for (int i = 0; i < kHalf; ++i) {
+    const uint64_t other = __shfl_xor_sync(0xFFFFFFFFu, V[i], D);
+    V[i] = fma2(V[i], (((i / C) / D) & 1) ? sr_neg : sr_pos, other);
+  }
+}
+
 // 1.5 * 2^23 + 8: adding it to |q| <= 7.5 rounds q to an integer k, half to
 // even, and leaves k + 8 (in 1..15) in the low four bits of the sum.
 constexpr float kMagic8 = 12582920.0f;
@@ -132,16 +151,9 @@ constexpr uint32_t kMagicBits = 0x4B400000u;   // bits of 1.5 * 2^23
 // Horner-packing eight sums (kMagicBits + n_e) as sum_e bits_e * 16^e leaves
 // this constant on top of the nibbles n_e (mod 2^32).
 constexpr uint32_t kHornerBias = kMagicBits * 0x11111111u;
-// The same for four sums per word in base 256 (one byte per code).
-constexpr uint32_t kHornerBias8 = kMagicBits * 0x01010101u;
-// Bytes n in 1..15 (code + 8) to the int8 codes n - 8, without borrows
-// between bytes: every byte is 0x81..0x8F before the subtraction.
-__device__ __forceinline__ uint32_t bytes_to_codes(uint32_t nb) {
-  return ((nb | 0x80808080u) - 0x08080808u) ^ 0x80808080u;
-}
 
-template <typename TIn, int G, int ACT, int OUT8>
-__global__ void __launch_bounds__(InTraits<TIn>::kMaxThreads, 1)
+template <typename TIn, int G, int ACT>
+__global__ void __maxnreg__(96)
     rotate_quant_pack_kernel(const TIn* __restrict__ x, int64_t M, int K, int64_t ldx, int rows_per_tile,
                              int nstages, int8_t* __restrict__ out, float* __restrict__ scale,
                              unsigned int* status) {
@@ -198,6 +210,11 @@ __global__ void __launch_bounds__(InTraits<TIn>::kMaxThreads, 1)
     }
   }
 
+  // sign of the two halves of V[i] in this lane's swizzle: chunks i / C and
+  // i / C + NCH / 2 (bit log2(NCH / 2) of the chunk index is outside L for
+  // fp32, inside it for bf16)
+  const bool hi_flip = (NCH / 2 < 8) && ((L >> 2) & 1);
+
   int it = 0;
   for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
     const int st = it % nstages;
@@ -206,7 +223,7 @@ __global__ void __launch_bounds__(InTraits<TIn>::kMaxThreads, 1)
     const bool valid = active && row < M && ok;
 
     // Slot chunk j (j < NCH/2) fills the low halves of V[C*j .. C*j+C), slot
-    // chunk j + NCH/2 the high halves: V[i] = (element i, element i + 64).
+    // chunk j + NCH/2 the high halves: V[i] = (element i, element i + 32).
     uint64_t V[kHalf];
     {
       const uint8_t* src = ring + st * stage_bytes + p * row_bytes + static_cast<size_t>(s) * kSlab * sizeof(TIn);
@@ -230,43 +247,30 @@ __global__ void __launch_bounds__(InTraits<TIn>::kMaxThreads, 1)
       }
     }
 
-    // Walsh-Hadamard butterflies: distances 1..32 on the pairs, 64 inside a pair.
+    // Walsh-Hadamard butterflies: distances 1..16 on the pairs, 32 inside a
+    // pair, then 64 and 128 across lanes.
     fht_stage2<1>(V);
     fht_stage2<2>(V);
     fht_stage2<4>(V);
     fht_stage2<8>(V);
     fht_stage2<16>(V);
-    fht_stage2<32>(V);
-    if (G >= 128) {
-#pragma unroll
-      for (int i = 0; i < kHalf; ++i) {
-        float a, b;
-        upk2(V[i], a, b);
-        V[i] = pk2(a + b, a - b);
-      }
-    }
-    if (G == 256) {
-      // Last stage across the two slabs of a group, held by lanes l and l^1
-      // (their swizzles L differ in bit 0, so chunk j carries the relative
-      // sign (-1)^j; both halves of V[i] lie in chunks of the same parity).
-      // Lower slab: a + b; upper slab: a - b.
-      const float ss = (s & 1) ? -1.0f : 1.0f;
-      const uint64_t ss2 = pk2(ss, ss);
-#pragma unroll
-      for (int i = 0; i < kHalf; ++i) {
-        const uint64_t other = __shfl_xor_sync(0xFFFFFFFFu, V[i], 1);
-        V[i] = ((i / C) & 1) ? sub2(mul2(V[i], ss2), other) : fma2(V[i], ss2, other);
-      }
-    }
-    float am[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int i = 0; i < kHalf; ++i) {
       float a, b;
       upk2(V[i], a, b);
-      am[i & 7] = fmaxf(am[i & 7], fmaxf(fabsf(a), fabsf(b)));
+      V[i] = pk2(a + b, a - b);
     }
-    const float amax = fmaxf(fmaxf(fmaxf(am[0], am[1]), fmaxf(am[2], am[3])),
-                             fmaxf(fmaxf(am[4], am[5]), fmaxf(am[6], am[7])));
+    if (G >= 128) fht_cross<1, C>(V, (s & 1) != 0);
+    if (G == 256) fht_cross<2, C>(V, (s & 2) != 0);
+
+    float am[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int i = 0; i < kHalf; ++i) {
+      float a, b;
+      upk2(V[i], a, b);
+      am[i & 3] = fmaxf(am[i & 3], fmaxf(fabsf(a), fabsf(b)));
+    }
+    const float amax = fmaxf(fmaxf(am[0], am[1]), fmaxf(am[2], am[3]));
     // max_k fl(|u_k| * norm) = fl(max_k |u_k| * norm): rounding is monotonic
     if (valid) atomicMax(&row_amax[it % 3][p], __float_as_uint(amax * norm));
     __syncthreads();   // every thread has its slab: ring slot st is free again
@@ -286,55 +290,31 @@ __global__ void __launch_bounds__(InTraits<TIn>::kMaxThreads, 1)
     const float amax_r = __uint_as_float(row_amax[it % 3][p]);
     const float sc = amax_r / 7.0f;   // fp32 division, as the method states
     if (s == 0) scale[row] = sc;
-    if (OUT8) {
-      // one int8 code per byte: words w and w + 16 take elements 4w..4w+3 and
-      // 64+4w..64+4w+3 (the low and high halves of V[4w .. 4w+4))
-      uint32_t codes[kSlab / 4];
-      if (sc > 0.0f) {
-        const float ni = norm * (1.0f / sc);
-        const uint64_t magic2 = pk2(kMagic8, kMagic8);
+    const float ni = sc > 0.0f ? norm * (1.0f / sc) : 0.0f;
+    const uint64_t magic2 = pk2(kMagic8, kMagic8);
+    // Quantiser multipliers per output chunk c of the low half: ni times the
+    // twist of chunk c -- the swizzle sign (-1)^popcount(c & L) and the rho
+    // factor of each shuffle stage; the high half (chunk c + NCH/2) adds the
+    // swizzle bit log2(NCH/2) when that bit lies inside L (bf16).
+    uint64_t mult[NCH / 2];
 #pragma unroll
-        for (int w = 0; w < kHalf / 4; ++w) {
-          uint32_t lo_acc = 0u, hi_acc = 0u;
-#pragma unroll
-          for (int e = 3; e >= 0; --e) {
-            const int i = 4 * w + e;
-            const float m = (__popc((i / C) & L) & 1) ? -ni : ni;
-            const uint64_t f = add2(mul2(V[i], pk2(m, m)), magic2);
-            float f0, f1;
-            upk2(f, f0, f1);
-            lo_acc = lo_acc * 256u + __float_as_uint(f0);
-            hi_acc = hi_acc * 256u + __float_as_uint(f1);
-          }
-          codes[w] = bytes_to_codes(lo_acc - kHornerBias8);
-          codes[w + kHalf / 4] = bytes_to_codes(hi_acc - kHornerBias8);
-        }
-      } else {
-#pragma unroll
-        for (int w = 0; w < kSlab / 4; ++w) codes[w] = 0u;
-      }
-      uint4* dst = reinterpret_cast<uint4*>(out + row * static_cast<int64_t>(K) + static_cast<int64_t>(s) * kSlab);
-#pragma unroll
-      for (int w = 0; w < kSlab / 16; ++w)
-        dst[w] = make_uint4(codes[4 * w], codes[4 * w + 1], codes[4 * w + 2], codes[4 * w + 3]);
-      continue;
+    for (int c = 0; c < NCH / 2; ++c) {
+      int par = __popc(c & L);
+      if (G >= 128) par += c & 1;
+      if (G == 256) par += (c >> 1) & 1;
+      const float m = (par & 1) ? -ni : ni;
+      mult[c] = pk2(m, hi_flip ? -m : m);
     }
-    uint32_t packed[kSlab / 8];
-    if (sc > 0.0f) {
-      const float ni = norm * (1.0f / sc);
-      const uint64_t magic2 = pk2(kMagic8, kMagic8);
-      // Pairs V[8w .. 8w+8) hold the codes of words w (low halves) and w + 8
-      // (high halves): quantise and Horner-pack them together, so only the
-      // sixteen words stay live next to the slab.
+    {
+      // words w and w + 4 take elements 8w..8w+7 and 32+8w..32+8w+7
+      uint32_t packed[kSlab / 8];
 #pragma unroll
       for (int w = 0; w < kHalf / 8; ++w) {
         uint32_t lo_acc = 0u, hi_acc = 0u;
 #pragma unroll
         for (int e = 7; e >= 0; --e) {
           const int i = 8 * w + e;
-          // sign of output chunk i / C (both halves share it, since L < 8)
-          const float m = (__popc((i / C) & L) & 1) ? -ni : ni;
-          const uint64_t f = add2(mul2(V[i], pk2(m, m)), magic2);
+          const uint64_t f = fma2(V[i], mult[i / C], magic2);
           float f0, f1;
           upk2(f, f0, f1);
           lo_acc = lo_acc * 16u + __float_as_uint(f0);
@@ -343,15 +323,11 @@ __global__ void __launch_bounds__(InTraits<TIn>::kMaxThreads, 1)
         packed[w] = (lo_acc - kHornerBias) ^ 0x88888888u;
         packed[w + kHalf / 8] = (hi_acc - kHornerBias) ^ 0x88888888u;
       }
-    } else {
-#pragma unroll
-      for (int w = 0; w < kSlab / 8; ++w) packed[w] = 0u;
+      uint4* dst = reinterpret_cast<uint4*>(out + row * static_cast<int64_t>(K / 2) +
+                                            static_cast<int64_t>(s) * (kSlab / 2));
+      dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+      dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
     }
-    uint4* dst = reinterpret_cast<uint4*>(out + row * static_cast<int64_t>(K / 2) +
-                                          static_cast<int64_t>(s) * (kSlab / 2));
-#pragma unroll
-    for (int w = 0; w < kSlab / 32; ++w)
-      dst[w] = make_uint4(packed[4 * w], packed[4 * w + 1], packed[4 * w + 2], packed[4 * w + 3]);
   }
   // After an abort, let every copy thread 0 issued land before the CTA exits.
   if (tid == 0 && abort_flag) {
@@ -362,65 +338,106 @@ __global__ void __launch_bounds__(InTraits<TIn>::kMaxThreads, 1)
   }
 }
 
-// Rows per tile and threads per CTA for a row of S slabs: as many whole rows
-// as fit in the thread limit (at most kMaxRows).
-static void rq_shape(int S, int max_threads, int* P, int* threads) {
-  int p = max_threads / S;
-  if (p < 1) p = 1;
-  if (p > kMaxRows) p = kMaxRows;
-  *P = p;
-  *threads = ((p * S + 31) / 32) * 32;
+// Registers per thread of one kernel instantiation (queried once).
+template <typename TIn, int G, int ACT>
+static int kernel_regs() {
+  static int regs = 0;
+  if (regs == 0) {
+    cudaFuncAttributes a;
+    regs = cudaFuncGetAttributes(&a, rotate_quant_pack_kernel<TIn, G, ACT>) == cudaSuccess && a.numRegs > 0
+               ? a.numRegs
+               : 128;
+  }
+  return regs;
 }
 
-template <typename TIn, int G, int ACT, int OUT8>
+struct RqPlan {
+  int P = 0, threads = 0, nst = 0;
+  int64_t grid = 0;
+};
+
+// Launch shape: rows per tile P, ring depth and grid.  Every row of S slabs
+// takes S threads; the CTAs that fit on an SM (registers, threads, ring
+// memory) run side by side, each on its own tiles.  The plan minimises the
+// estimated time of the busiest SM: the rows it holds, divided by the warps
+// that share them (up to 16, beyond which an SM is saturated) and by the
+// fraction of lanes that carry a slab.
+static RqPlan plan_rq(int64_t M, int K, size_t elem_bytes, int regs, int num_sms) {
+  const int S = K / kSlab;
+  const size_t row_bytes = static_cast<size_t>(K) * elem_bytes;
+  const int regs_warp = (regs * 32 + 255) / 256 * 256;
+  RqPlan best;
+  double best_t = 1e30;
+  const int pmax = kMaxThreads / S < kMaxRows ? kMaxThreads / S : kMaxRows;
+  for (int P = 1; P <= pmax; ++P) {
+    const int threads = (P * S + 31) / 32 * 32;
+    const int warps = threads / 32;
+    int cps = 65536 / (warps * regs_warp);
+    if (2048 / threads < cps) cps = 2048 / threads;
+    if (cps > 8) cps = 8;
+    const int64_t tiles = (M + P - 1) / P;
+    for (int c = 1; c <= cps; ++c) {
+      int nst = static_cast<int>(kRingBytesPerSm / (static_cast<size_t>(c) * P * row_bytes));
+      if (nst > kMaxStages) nst = kMaxStages;
+      if (nst < kMinStages) break;
+      const int64_t grid = tiles < static_cast<int64_t>(num_sms) * c ? tiles : static_cast<int64_t>(num_sms) * c;
+      const int64_t per_cta = (tiles + grid - 1) / grid;
+      const int64_t ctas_sm = (grid + num_sms - 1) / num_sms;
+      const double sm_rows = static_cast<double>(per_cta * P * ctas_sm);
+      const double w = static_cast<double>(warps * ctas_sm) < 16.0 ? static_cast<double>(warps * ctas_sm) : 16.0;
+      const double eff = static_cast<double>(P * S) / threads;
+      const double t = sm_rows / (w * eff) * (1.0 + 0.02 * (kMaxStages - nst));
+      if (t < best_t - 1e-9) {
+        best_t = t;
+        best.P = P;
+        best.threads = threads;
+        best.nst = nst;
+        best.grid = grid;
+      }
+    }
+  }
+  return best;
+}
+
+template <typename TIn, int G, int ACT>
 static cudaError_t launch_rq(const TIn* x, int64_t M, int K, int64_t ldx, int8_t* out, float* scale, int num_sms,
                              unsigned int* status, cudaStream_t stream) {
   const int S = K / kSlab;
-  if (S > InTraits<TIn>::kMaxThreads) return cudaErrorInvalidValue;
-  int P, threads;
-  rq_shape(S, InTraits<TIn>::kMaxThreads, &P, &threads);
-  const size_t stage_bytes = static_cast<size_t>(P) * K * sizeof(TIn);
-  int nst = static_cast<int>(kRingBytes / stage_bytes);
-  if (nst > kMaxStages) nst = kMaxStages;
-  if (nst < 1) return cudaErrorInvalidValue;
-  const size_t smem = nst * stage_bytes;
-  auto kern = rotate_quant_pack_kernel<TIn, G, ACT, OUT8>;
+  if (S < 1 || S > kMaxThreads) return cudaErrorInvalidValue;
+  const RqPlan pl = plan_rq(M, K, sizeof(TIn), kernel_regs<TIn, G, ACT>(), num_sms);
+  if (pl.P < 1) return cudaErrorInvalidValue;
+  const size_t smem = static_cast<size_t>(pl.nst) * pl.P * K * sizeof(TIn);
+  auto kern = rotate_quant_pack_kernel<TIn, G, ACT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  const int64_t tiles = (M + P - 1) / P;
-  const int64_t grid = tiles < num_sms ? tiles : num_sms;
-  kern<<<static_cast<unsigned>(grid), threads, smem, stream>>>(x, M, K, ldx, P, nst, out, scale, status);
+  kern<<<static_cast<unsigned>(pl.grid), pl.threads, smem, stream>>>(x, M, K, ldx, pl.P, pl.nst, out, scale,
+                                                                      status);
   return cudaGetLastError();
 }
 
-template <typename TIn, int OUT8>
+template <typename TIn>
 static cudaError_t dispatch_rq(const TIn* x, int64_t M, int K, int64_t ldx, int g, int act, int8_t* out,
                                float* scale, int num_sms, unsigned int* status, cudaStream_t stream) {
   if (act == 0) {
-    if (g == 64) return launch_rq<TIn, 64, 0, OUT8>(x, M, K, ldx, out, scale, num_sms, status, stream);
-    if (g == 128) return launch_rq<TIn, 128, 0, OUT8>(x, M, K, ldx, out, scale, num_sms, status, stream);
-    if (g == 256) return launch_rq<TIn, 256, 0, OUT8>(x, M, K, ldx, out, scale, num_sms, status, stream);
+    if (g == 64) return launch_rq<TIn, 64, 0>(x, M, K, ldx, out, scale, num_sms, status, stream);
+    if (g == 128) return launch_rq<TIn, 128, 0>(x, M, K, ldx, out, scale, num_sms, status, stream);
+    if (g == 256) return launch_rq<TIn, 256, 0>(x, M, K, ldx, out, scale, num_sms, status, stream);
   } else {
-    if (g == 64) return launch_rq<TIn, 64, 1, OUT8>(x, M, K, ldx, out, scale, num_sms, status, stream);
-    if (g == 128) return launch_rq<TIn, 128, 1, OUT8>(x, M, K, ldx, out, scale, num_sms, status, stream);
-    if (g == 256) return launch_rq<TIn, 256, 1, OUT8>(x, M, K, ldx, out, scale, num_sms, status, stream);
+    if (g == 64) return launch_rq<TIn, 64, 1>(x, M, K, ldx, out, scale, num_sms, status, stream);
+    if (g == 128) return launch_rq<TIn, 128, 1>(x, M, K, ldx, out, scale, num_sms, status, stream);
+    if (g == 256) return launch_rq<TIn, 256, 1>(x, M, K, ldx, out, scale, num_sms, status, stream);
   }
   return cudaErrorInvalidValue;
 }
 
 cudaError_t rotate_quant_bf16(const uint16_t* x, int64_t M, int K, int64_t ldx, int g, int act, int8_t* out,
                               float* scale, int num_sms, unsigned int* status, cudaStream_t stream) {
-  return dispatch_rq<uint16_t, 0>(x, M, K, ldx, g, act, out, scale, num_sms, status, stream);
-}
-
-cudaError_t rotate_quant_bf16_i8(const uint16_t* x, int64_t M, int K, int64_t ldx, int g, int act, int8_t* out,
-                                 float* scale, int num_sms, unsigned int* status, cudaStream_t stream) {
-  return dispatch_rq<uint16_t, 1>(x, M, K, ldx, g, act, out, scale, num_sms, status, stream);
+  return dispatch_rq<uint16_t>(x, M, K, ldx, g, act, out, scale, num_sms, status, stream);
 }
 
 cudaError_t rotate_quant_f32(const float* x, int64_t M, int K, int64_t ldx, int g, int8_t* out, float* scale,
                              int num_sms, unsigned int* status, cudaStream_t stream) {
-  return dispatch_rq<float, 0>(x, M, K, ldx, g, 0, out, scale, num_sms, status, stream);
+  return dispatch_rq<float>(x, M, K, ldx, g, 0, out, scale, num_sms, status, stream);
 }
 
 }  // namespace w4a4

@@ -26,16 +26,13 @@ int validate_linear(const int8_t* Xq, const float* sx, const int8_t* Wq, const f
 // ---- activation / weight rotate + quantise + pack (quant.cu)
 cudaError_t rotate_quant_bf16(const uint16_t* x, int64_t M, int K, int64_t ldx, int g, int act, int8_t* out,
                               float* scale, int num_sms, unsigned int* status, cudaStream_t stream);
-// Same rotation and quantisation, every code stored as one int8 ([M, K] bytes).
-cudaError_t rotate_quant_bf16_i8(const uint16_t* x, int64_t M, int K, int64_t ldx, int g, int act, int8_t* out,
-                                 float* scale, int num_sms, unsigned int* status, cudaStream_t stream);
 cudaError_t rotate_quant_f32(const float* x, int64_t M, int K, int64_t ldx, int g, int8_t* out, float* scale,
                              int num_sms, unsigned int* status, cudaStream_t stream);
-// Largest K the in-register rotate kernel supports (one row per CTA at most):
-// 256 threads x 128 codes for bf16 rows, 192 threads x 128 codes for fp32
-// rows (weights).
-constexpr int kQuantMaxK = 256 * 128;
-constexpr int kQuantMaxKF32 = 192 * 128;
+// Largest K the in-register rotate kernel supports: 512 threads x 64 codes
+// per row for bf16 rows; fp32 rows (weights) are limited by two ring stages
+// of one row in shared memory (2 x 96 KB).
+constexpr int kQuantMaxK = 512 * 64;
+constexpr int kQuantMaxKF32 = 384 * 64;
 
 // ---- tcgen05 GEMM (gemm.cu)
 struct GemmArgs {
@@ -56,16 +53,6 @@ cudaError_t gemm_tc_launch(const CUtensorMap& tmA, const CUtensorMap& tmB, const
                            int num_sms, cudaStream_t stream);
 constexpr int kGemmBM = 256;
 constexpr int kGemmBN = 256;
-
-// ---- tcgen05 GEMM with the weights widened into tensor memory (gemm_ts.cu)
-// tmAct: activation codes, one int8 per byte [M, K], box {128 bytes, 96 rows},
-// 128-byte swizzle; tmW: packed weights [N, K/2] bytes, box {64 bytes, 128
-// rows}, 64-byte swizzle; tmY: bf16 output [M, N] (row stride ldo), box
-// {32, 32}, no swizzle (unused for int32 output).  Clusters of 2 CTAs.
-cudaError_t gemm_ts_launch(const CUtensorMap& tmAct, const CUtensorMap& tmW, const CUtensorMap& tmY,
-                           const GemmArgs& a, int num_sms, cudaStream_t stream);
-constexpr int kTsTileW = 256;   // weight rows per cluster tile
-constexpr int kTsTileA = 192;   // activation rows per cluster tile
 
 // ---- small-M weight-streaming GEMM (smallm.cu)
 struct SmallMArgs {
