@@ -250,6 +250,47 @@ def time_loop(fn, steps, stream):
     return start.elapsed_time(end) / 1e3    # seconds
 
 
+class GraphLoop:
+    """`steps` calls of fn(i) recorded once into CUDA graphs (chunks of at
+    most 200 calls) and replayed: the GPU runs the same kernels with the same
+    arguments as the eager loop, without the host's per-call launch work.
+    Capture and replay use a side stream of their own (capture cannot use the
+    default stream); fn runs there eagerly twice first, so that everything it
+    sets up per stream exists before the capture."""
+
+    def __init__(self, fn, steps):
+        chunk = steps if steps <= 200 else next(c for c in (200, 100, 50, 40, 25, 20, 10, 8, 5, 4, 2, 1)
+                                                if steps % c == 0)
+        self.graph = torch.cuda.CUDAGraph()
+        self.reps = steps // chunk
+        self.stream = torch.cuda.Stream()
+        torch.cuda.synchronize()
+        with torch.cuda.stream(self.stream):
+            fn(0)
+            fn(1)
+            self.stream.synchronize()
+            with torch.cuda.graph(self.graph, stream=self.stream):
+                for i in range(chunk):
+                    fn(i)
+        self.stream.synchronize()
+
+    def run(self):
+        with torch.cuda.stream(self.stream):
+            for _ in range(self.reps):
+                self.graph.replay()
+
+
+def time_graph(loop):
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    start.record(loop.stream)
+    loop.run()
+    end.record(loop.stream)
+    end.synchronize()
+    return start.elapsed_time(end) / 1e3    # seconds
+
+
 def run_impl(args, cfg, world, rank, local):
     import w4a4_hadamard_rotated_b200 as w4
     w4.load_library()
@@ -262,19 +303,26 @@ def run_impl(args, cfg, world, rank, local):
         s = sets[i % len(sets)]
         w4.linear_fused(s["x"], s["Wq"], s["sw"], s["b"], g, cfg.act, out=s["y"])
 
-    # ---- the timed region: exactly `steps` fused layer calls
-    sampler = ClockSampler(device.index) if rank == 0 else None
-    if sampler:
-        sampler.start()
+    # ---- the timed region: exactly `steps` fused layer calls, replayed from
+    # CUDA graphs (the eager loop's time, host launch work included, is
+    # reported beside it)
     for i in range(args.warmup):
         fused(i)
     torch.cuda.synchronize()
+    loop = GraphLoop(fused, args.steps)
+    loop.run()   # one untimed replay
+    sampler = ClockSampler(device.index) if rank == 0 else None
+    if sampler:
+        sampler.start()
+    torch.cuda.synchronize()
     barrier(world)
-    dt = time_loop(fused, args.steps, stream)
+    dt = time_graph(loop)
     torch.cuda.synchronize()
     barrier(world)
     clocks = sampler.stop() if sampler else None
     dt_max = max_over_ranks(dt, world)
+    del loop
+    dt_eager = max_over_ranks(time_loop(fused, args.steps, stream), world)
     ops = float(cfg.ops())
     value = world * ops * args.steps / dt_max / 1e12
     ms_per_step = dt_max / args.steps * 1e3
@@ -292,14 +340,14 @@ def run_impl(args, cfg, world, rank, local):
         w4.linear(s["Xq"], s["sx"], s["Wq"], s["sw"], s["b"], out=s["y"])
 
 
-    reps = max(min(args.steps, 2000), 20)
+    reps = 200
     for i in range(3):
         quant(i)
         gemm(i)
-    t_quant = time_loop(quant, reps, stream) / reps
+    t_quant = time_graph(GraphLoop(quant, reps)) / reps
     for i in range(len(sets)):
         quant(i)
-    t_gemm = time_loop(gemm, reps, stream) / reps
+    t_gemm = time_graph(GraphLoop(gemm, reps)) / reps
 
     # ---- end to end through the public API with host buffers: pinned x in,
     # y out, copies inside the timed region
@@ -358,8 +406,10 @@ def run_impl(args, cfg, world, rank, local):
         "config": {"workload": cfg.name, "M": cfg.M, "K": cfg.K, "N": cfg.N, "g": cfg.g, "bias": cfg.bias,
                    "gelu_input": bool(cfg.act),
                    "l2": f"{len(sets)} rotating input/weight/output sets (> 2x L2)",
+                   "launch": "CUDA graphs of the fused calls, replayed",
                    "parallelism": f"replicas x{world}"},
         "us_per_layer": ms_per_step * 1e3,
+        "us_per_layer_eager_launches": dt_eager / args.steps * 1e6,
         "roofline_fraction_of_layer": roof_time / (ms_per_step / 1e3),
         "layer_roofline_us": roof_time * 1e6,
         "kernels_us": {"rotate_quant_pack": t_quant * 1e6, ("smallm" if small else "gemm_tc"): t_gemm * 1e6},

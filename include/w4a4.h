@@ -16,8 +16,7 @@
  *
  * Conventions for every entry point:
  *   - Every tensor pointer is DEVICE memory owned by the caller; the library
- *     never allocates or frees memory (w4a4_linear_noalloc uses a fixed array
- *     of the library's own device memory instead of a caller workspace).  Matrices are row-major with the
+ *     never allocates or frees memory.  Matrices are row-major with the
  *     inner dimension contiguous; ld* arguments are row strides in elements.
  *   - bf16 tensors are passed as raw 16-bit patterns (uint16_t).
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  All work is
@@ -93,13 +92,11 @@ int w4a4_quantize_activation(const uint16_t* x, int64_t M, int64_t K, int64_t ld
  *   bias [N] bf16 bits or NULL
  *   y  [M, N] bf16 bits output, row stride ldy >= N, ldy % 8 == 0, 16-byte aligned
  *   M >= 0, N >= 1, N % 8 == 0, 32 <= K <= 131072, K % 32 == 0; Xq/Wq 16-byte aligned
- *   workspace: device scratch of at least w4a4_workspace_bytes(M, N, K)
- *       bytes, 256-byte aligned (may be NULL when that size is 0).  Its first
- *       32 KiB (arrival counters of the small-M kernel) must be zero before the
- *       first call; every call leaves them zero.  Calls that share one
- *       workspace must be ordered on the same stream.
- * M <= 64 takes the weight-streaming split-K kernel, larger M the tcgen05
- * tensor-core kernel; both give bit-identical int32 accumulators.
+ *   workspace, workspace_bytes: reserved; no kernel needs scratch memory
+ *       (w4a4_workspace_bytes returns 0), so both may be NULL / 0.
+ * M <= 64 takes the weight-streaming split-K kernel (K slices reduced on chip
+ * within a CTA cluster), larger M the tcgen05 tensor-core kernel; both give
+ * bit-identical int32 accumulators.
  */
 int w4a4_linear(const int8_t* Xq, const float* sx, const int8_t* Wq, const float* sw,
                 const uint16_t* bias, uint16_t* y, int64_t M, int64_t N, int64_t K,
@@ -109,17 +106,18 @@ int w4a4_linear(const int8_t* Xq, const float* sx, const int8_t* Wq, const float
  * Fused layer: w4a4_quantize_activation followed by w4a4_linear, with the
  * packed activation and its scales kept in the workspace.
  *   x [M, K] bf16 bits with row stride ldx; other arguments as above.
- *   workspace: at least w4a4_fused_workspace_bytes(M, N, K) bytes, laid out as
- *       [small-M scratch, counter block first][quantised x][sx]; the same rule
- *       for its first 32 KiB holds, so one zero-filled buffer can serve both
- *       w4a4_linear and w4a4_linear_fused calls of any shape.
+ *   workspace: at least w4a4_fused_workspace_bytes(M, N, K) bytes, 256-byte
+ *       aligned, laid out as [packed x][sx]; its contents need no
+ *       initialisation.  Calls that share one workspace must be ordered on the
+ *       same stream.
  */
 int w4a4_linear_fused(const uint16_t* x, int64_t ldx, const int8_t* Wq, const float* sw,
                       const uint16_t* bias, uint16_t* y, int64_t ldy, int64_t M, int64_t N,
                       int64_t K, int g, int act, void* workspace, size_t workspace_bytes,
                       void* stream);
 
-/* Workspace sizes in bytes (0 when none is needed).  Pure host functions. */
+/* Workspace sizes in bytes (0 when none is needed: w4a4_workspace_bytes is
+ * always 0).  Pure host functions. */
 size_t w4a4_workspace_bytes(int64_t M, int64_t N, int64_t K);
 size_t w4a4_fused_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
@@ -143,17 +141,11 @@ int w4a4_gemm_s32(const int8_t* Xq, const int8_t* Wq, int32_t* acc, int64_t M, i
  * that must not call cudaMalloc after start-up (an allocation can
  * synchronise the device and fragment a pool sized in advance).
  *   Arguments, layouts and results are those of w4a4_linear; the output is
- *   bit-identical to it.  Scratch (split-K partial tiles and arrival
- *   counters) lives in a fixed 4 MiB array of this library's own device
- *   memory, which every GPU that loads the library keeps until the process
- *   exits; a shape whose scratch, w4a4_workspace_bytes(M, N, K), exceeds
- *   4 MiB is rejected with W4A4_ERR_WORKSPACE before anything is launched
- *   (M > 64 or N > 1048576 gives W4A4_ERR_SHAPE).
- *   The first call on a device resolves the array's device address and
- *   clears its counter block on `stream`; make that first call before any
- *   stream capture.  Every call uses the same array and leaves the counters
- *   at zero; calls that may overlap on the GPU (other streams, other host
- *   threads) race on the array and must be serialised by the caller.
+ *   bit-identical to it.  The small-M kernel reduces its K slices in the
+ *   shared memory of a CTA cluster, so no scratch memory of any kind is
+ *   used: neither a caller workspace nor memory of the library's own.
+ *   M > 64 gives W4A4_ERR_SHAPE before anything is launched.  Calls are
+ *   independent (they may overlap on the GPU).
  */
 int w4a4_linear_noalloc(const int8_t* Xq, const float* sx, const int8_t* Wq, const float* sw,
                         const uint16_t* bias, uint16_t* y, int64_t M, int64_t N, int64_t K, int64_t ldy,

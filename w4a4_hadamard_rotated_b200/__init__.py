@@ -101,10 +101,8 @@ def _bits(t):
     return t.view(torch.int16)
 
 
-# Workspaces are cached per (purpose, device, stream) and grown on demand.  The
-# small-M kernel needs its workspace zero-filled once and keeps it zero itself,
-# so the fused entry (whose workspace starts with the packed activation) gets
-# a buffer of its own.
+# Workspaces (the fused entry's packed activation and scales) are cached per
+# (purpose, device, stream) and grown on demand.
 _workspaces = {}
 
 
@@ -113,7 +111,7 @@ def workspace(nbytes, device, kind="linear"):
            torch.cuda.current_stream(device).cuda_stream)
     buf = _workspaces.get(key)
     if buf is None or buf.numel() < nbytes:
-        buf = torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+        buf = torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
         _workspaces[key] = buf
     return buf
 
@@ -188,18 +186,14 @@ def gemm_s32(Xq, Wq, path=0, out=None):
     N = Wq.shape[0]
     K = 2 * Kh
     acc = out if out is not None else torch.empty(M, N, dtype=torch.int32, device=Xq.device)
-    nbytes = lib.w4a4_workspace_bytes(M, N, K) if path == 1 else 0
-    if path == 1 and nbytes == 0 and M > 0:
-        raise ValueError("path 1 (small-M kernel) needs M <= the small-M threshold")
-    ws = workspace(nbytes, Xq.device) if nbytes else None
-    _check(lib.w4a4_gemm_s32(_ptr(Xq), _ptr(Wq), _ptr(acc), M, N, K, acc.stride(0), path, _ptr(ws), nbytes,
+    _check(lib.w4a4_gemm_s32(_ptr(Xq), _ptr(Wq), _ptr(acc), M, N, K, acc.stride(0), path, None, 0,
                              _stream(Xq)), "w4a4_gemm_s32")
     return acc
 
 
 def linear_noalloc(Xq, sx, Wq, sw, bias=None, out=None):
-    """Small-M (M <= 64) linear with no workspace: the library's own fixed
-    scratch array stands in for it (see w4a4_linear_noalloc in the header)."""
+    """Small-M (M <= 64) linear that takes no workspace and uses no scratch
+    memory (see w4a4_linear_noalloc in the header)."""
     lib = load_library()
     _need_cuda(Xq, torch.int8, "Xq")
     _need_cuda(Wq, torch.int8, "Wq")

@@ -75,8 +75,10 @@ EncodeTiledFn encode_fn() {
 }  // namespace
 
 // 2-D map over a packed int4 matrix [rows, K/2] bytes, box {64 bytes, box_rows};
-// out-of-range rows and columns read as zero.
-int packed_map(CUtensorMap* map, const int8_t* base, int64_t rows, int64_t K, int box_rows) {
+// out-of-range rows and columns read as zero.  swizzle64: the box lands in
+// shared memory with the 64-byte swizzle (16-byte chunk j of row r at
+// j ^ ((r >> 1) & 3)), for readers that take one row per thread.
+int packed_map(CUtensorMap* map, const int8_t* base, int64_t rows, int64_t K, int box_rows, bool swizzle64) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return W4A4_ERR_CUDA;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(rows)};
@@ -84,8 +86,8 @@ int packed_map(CUtensorMap* map, const int8_t* base, int64_t rows, int64_t K, in
   const cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(box_rows)};
   const cuuint32_t estr[2] = {1u, 1u};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? W4A4_OK : W4A4_ERR_CUDA;
 }
 
@@ -142,18 +144,14 @@ int check_gemm_shape(int64_t M, int64_t N, int64_t K) {
 // Shared body of w4a4_linear / w4a4_gemm_s32 after validation.  path 0: the
 // tcgen05 tensor-core kernel; 1: the small-M weight-streaming kernel.
 int run_linear(const int8_t* Xq, const float* sx, const int8_t* Wq, const float* sw, const uint16_t* bias, void* out,
-               int64_t M, int64_t N, int64_t K, int64_t ldo, int out_s32, int path, void* ws, size_t ws_bytes,
-               cudaStream_t stream) {
+               int64_t M, int64_t N, int64_t K, int64_t ldo, int out_s32, int path, cudaStream_t stream) {
   DeviceInfo* dev = nullptr;
   int st = current_device(&dev);
   if (st != W4A4_OK) return st;
   if (M == 0) return W4A4_OK;
   if (path == 1) {
-    if (N > kSmallMMaxN) return W4A4_ERR_SHAPE;
-    const size_t need = smallm_workspace_bytes(M, N, K);
-    if (ws == nullptr || ws_bytes < need || !aligned(ws, 256)) return W4A4_ERR_WORKSPACE;
     CUtensorMap tmW, tmX;
-    if ((st = packed_map(&tmW, Wq, N, K, 128)) != W4A4_OK) return st;
+    if ((st = packed_map(&tmW, Wq, N, K, 128, true)) != W4A4_OK) return st;
     if ((st = packed_map(&tmX, Xq, M, K, smallm_rows_padded(M))) != W4A4_OK) return st;
     SmallMArgs a{};
     a.xq = Xq;
@@ -167,10 +165,8 @@ int run_linear(const int8_t* Xq, const float* sx, const int8_t* Wq, const float*
     a.out = out;
     a.ldo = ldo;
     a.out_s32 = out_s32;
-    a.counters = static_cast<unsigned int*>(ws);
-    a.partial = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + kSmallMCounterBytes);
     a.status = dev->status;
-    return smallm_launch_tm(tmW, tmX, a, dev->num_sms, stream) == cudaSuccess ? W4A4_OK : W4A4_ERR_CUDA;
+    return smallm_launch_tm(tmW, tmX, a, stream) == cudaSuccess ? W4A4_OK : W4A4_ERR_CUDA;
   }
   CUtensorMap tmA, tmB, tmY;
   if ((st = packed_map(&tmA, Xq, M, K, kGemmBM / 2)) != W4A4_OK) return st;
@@ -287,28 +283,24 @@ int w4a4_quantize_activation(const uint16_t* x, int64_t M, int64_t K, int64_t ld
              : W4A4_ERR_CUDA;
 }
 
+// No kernel of the linear needs a workspace any more (the small-M kernel
+// reduces its K slices on chip); the workspace arguments of w4a4_linear and
+// w4a4_gemm_s32 are kept for ABI stability and may be NULL.
 size_t w4a4_workspace_bytes(int64_t M, int64_t N, int64_t K) {
-  if (M <= 0 || N <= 0 || K <= 0) return 0;
-  if (M <= smallm_threshold()) return smallm_workspace_bytes(M, N, K);
+  (void)M;
+  (void)N;
+  (void)K;
   return 0;
 }
 
-// The fused workspace always starts with the small-M counter block (even when
-// this shape takes the large-M kernel), so that the block stays at offset 0 and
-// stays zero whatever shapes share the buffer.
-static size_t fused_linear_part(int64_t M, int64_t N, int64_t K) {
-  const size_t lin = w4a4_workspace_bytes(M, N, K);
-  return round256(lin > kSmallMCounterBytes ? lin : kSmallMCounterBytes);
-}
-
-// Bytes of the packed activation in the fused workspace.
+// The fused workspace holds the packed activation and its scales.
 static size_t fused_codes_bytes(int64_t M, int64_t K) {
   return round256(static_cast<size_t>(M) * static_cast<size_t>(K / 2));
 }
 
 size_t w4a4_fused_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   if (M <= 0 || N <= 0 || K <= 0) return 0;
-  return fused_linear_part(M, N, K) + fused_codes_bytes(M, K) + round256(static_cast<size_t>(M) * 4);
+  return fused_codes_bytes(M, K) + round256(static_cast<size_t>(M) * 4);
 }
 
 int w4a4_linear(const int8_t* Xq, const float* sx, const int8_t* Wq, const float* sw, const uint16_t* bias,
@@ -317,8 +309,9 @@ int w4a4_linear(const int8_t* Xq, const float* sx, const int8_t* Wq, const float
   int st = validate_linear(Xq, sx, Wq, sw, bias, y, M, N, K, ldy, 0);
   if (st != W4A4_OK) return st;
   const int path = (M <= smallm_threshold()) ? 1 : 0;
-  return run_linear(Xq, sx, Wq, sw, bias, y, M, N, K, ldy, 0, path, workspace, workspace_bytes,
-                    static_cast<cudaStream_t>(stream));
+  (void)workspace;
+  (void)workspace_bytes;
+  return run_linear(Xq, sx, Wq, sw, bias, y, M, N, K, ldy, 0, path, static_cast<cudaStream_t>(stream));
 }
 
 int w4a4_gemm_s32(const int8_t* Xq, const int8_t* Wq, int32_t* acc, int64_t M, int64_t N, int64_t K, int64_t ldc,
@@ -327,8 +320,9 @@ int w4a4_gemm_s32(const int8_t* Xq, const int8_t* Wq, int32_t* acc, int64_t M, i
   if (st != W4A4_OK) return st;
   if (path != 0 && path != 1) return W4A4_ERR_ARG;
   if (path == 1 && M > kSmallMMax) return W4A4_ERR_SHAPE;
-  return run_linear(Xq, nullptr, Wq, nullptr, nullptr, acc, M, N, K, ldc, 1, path, workspace, workspace_bytes,
-                    static_cast<cudaStream_t>(stream));
+  (void)workspace;
+  (void)workspace_bytes;
+  return run_linear(Xq, nullptr, Wq, nullptr, nullptr, acc, M, N, K, ldc, 1, path, static_cast<cudaStream_t>(stream));
 }
 
 int w4a4_linear_fused(const uint16_t* x, int64_t ldx, const int8_t* Wq, const float* sw, const uint16_t* bias,
@@ -351,16 +345,14 @@ int w4a4_linear_fused(const uint16_t* x, int64_t ldx, const int8_t* Wq, const fl
   }
   const size_t need = w4a4_fused_workspace_bytes(M, N, K);
   if (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 256)) return W4A4_ERR_WORKSPACE;
-  // Layout: [linear workspace, counter block first][quantised x][sx], so that
-  // the counter block sits at offset 0 for every shape and every entry point.
+  // Layout: [packed x][sx]
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  const size_t lin_bytes = fused_linear_part(M, N, K);
-  int8_t* xq = reinterpret_cast<int8_t*>(ws + lin_bytes);
-  float* sx = reinterpret_cast<float*>(ws + lin_bytes + fused_codes_bytes(M, K));
+  int8_t* xq = reinterpret_cast<int8_t*>(ws);
+  float* sx = reinterpret_cast<float*>(ws + fused_codes_bytes(M, K));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if ((st = w4a4_quantize_activation(x, M, K, ldx, g, act, xq, sx, stream)) != W4A4_OK) return st;
   const int path = (M <= smallm_threshold()) ? 1 : 0;
-  return run_linear(xq, sx, Wq, sw, bias, y, M, N, K, ldy, 0, path, ws, lin_bytes, s);
+  return run_linear(xq, sx, Wq, sw, bias, y, M, N, K, ldy, 0, path, s);
 }
 
 int w4a4_last_device_error(void* stream) {

@@ -11,15 +11,24 @@
 //   * The MMA M side is 128 weight rows, the N side the activation rows padded
 //     to NP in {16, 32, 64}; tcgen05.mma.kind::i8 accumulates int32 in TMEM.
 //   * Work units are (128-row weight tile, K slice) pairs, sized so that about
-//     two CTAs run on every SM; each streams its weight slice through a TMA
-//     ring, widens nibbles to bytes in shared memory and issues the MMAs.
-//   * K slices are reduced exactly: each CTA stores its int32 partial tile in
-//     its own workspace slot, then increments a per-tile arrival counter with
-//     a wrapping atomicInc; the CTA that arrives last sums the slots in split
-//     order (integer addition, so the result is exact and deterministic),
-//     applies the epilogue and writes y.  The wrap leaves every counter at 0,
-//     so only the counter block has to be zero before the first call.  With a
-//     single K slice the epilogue runs directly from the accumulator.
+//     two CTAs run on every SM.  One thread issues the TMA loads of all the
+//     CTA's k-blocks at once (an 8-deep ring), so every SM keeps tens of KB of
+//     weight reads in flight from the first cycle.
+//   * Widening the weights in shared memory would cost six bytes of
+//     shared-memory traffic per streamed byte, more than an SM sustains at
+//     HBM rate; so four warps widen each packed weight row (one thread per
+//     row, read from a 64-byte-swizzled tile) into tensor memory with
+//     tcgen05.st, and the MMA reads its A operand from there.  The few
+//     activation rows are widened into shared memory (the B operand).  Each
+//     nibble q becomes the byte 16*q (no sign extension) in the byte order
+//     (1,3,5,7, 0,2,4,6) for both operands, so the MMA accumulates 256*acc.
+//   * The K slices of one weight tile run as one cluster of up to 8 CTAs.
+//     Each CTA parks its int32 partial tile in its shared memory; after a
+//     cluster barrier, CTA c reads its share of the tile's rows from every
+//     CTA of the cluster (distributed shared memory), sums them in rank order
+//     (integer addition: exact and deterministic), applies the epilogue and
+//     writes y.  The reduction never leaves the chip, and the kernel needs no
+//     workspace.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -34,66 +43,76 @@ namespace {
 constexpr int WM = 128;        // weight rows per tile (MMA M)
 constexpr int BK = 128;        // codes per k-block
 constexpr int BKP = BK / 2;    // packed bytes per k-block row
-constexpr int SP = 3;          // packed ring depth
-constexpr int SWD = 2;         // widened ring depth
-constexpr int kWorkWarps = 4;  // widen + epilogue warps
-constexpr int kThreads = (2 + kWorkWarps) * 32;
+constexpr int SP = 8;          // packed ring depth (loads in flight per CTA), at most
+constexpr int ST = 6;          // widened stages (weights in tensor memory, activations in shared memory), at most
+constexpr int kWorkWarps = 4;  // widen + epilogue warps, one per tensor-memory lane quarter
+constexpr int kGroups = 2;     // widen groups of kWorkWarps warps, taking turns by k-block
+constexpr int kThreads = (2 + kGroups * kWorkWarps) * 32;
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kTmemA = 64;   // first widened-weight column (the accumulator takes NP <= 64)
 
+// Two CTAs share an SM, so each keeps its rings within ~110 KB of shared
+// memory: NP = 64 (8 KB widened activations per stage) takes shallower rings.
 template <int NP>
 struct Layout {
-  static constexpr uint32_t kWideW = WM * BK;     // 16 KB
-  static constexpr uint32_t kWideX = NP * BK;     // <= 8 KB
+  static constexpr int kSP = NP == 64 ? 6 : SP;
+  static constexpr int kST = NP == 64 ? 4 : ST;
   static constexpr uint32_t kPackW = WM * BKP;    // 8 KB
   static constexpr uint32_t kPackX = NP * BKP;    // <= 4 KB
-  static constexpr uint32_t kOffWideW = 0;
-  static constexpr uint32_t kOffWideX = kOffWideW + SWD * kWideW;
-  static constexpr uint32_t kOffPackW = kOffWideX + SWD * kWideX;
-  static constexpr uint32_t kOffPackX = kOffPackW + SP * kPackW;
-  static constexpr uint32_t kBytes = kOffPackX + SP * kPackX;
+  static constexpr uint32_t kWideX = NP * BK;     // <= 8 KB
+  static constexpr uint32_t kOffWideX = 0;        // 1024-aligned stages (128-byte swizzle)
+  static constexpr uint32_t kOffPackW = kOffWideX + kST * kWideX;   // 1024-aligned (64-byte swizzle)
+  static constexpr uint32_t kOffPackX = kOffPackW + kSP * kPackW;
+  static constexpr uint32_t kBytes = kOffPackX + kSP * kPackX;
   static constexpr uint32_t kAlloc = kBytes + 1024;
-  static constexpr uint32_t kTmemCols = NP < 32 ? 32 : NP;
+  static_assert(kOffPackW % 1024 == 0, "alignment");
 };
 
 struct Bars {
-  uint64_t packed_full[SP];
-  uint64_t packed_empty[SP];
-  uint64_t wide_full[SWD];
-  uint64_t wide_empty[SWD];
+  float sx[64];          // activation scales (epilogue operands, staged early)
+  float sw[WM];          // this tile's weight scales
+  float bias[WM];        // this tile's bias (fp32)
+  uint64_t full[SP];     // TMA transaction barrier (weights + activations of one k-block)
+  uint64_t empty[SP];    // kWorkWarps arrivals (packed data read)
+  uint64_t wfull[ST];    // kWorkWarps arrivals (widened stage written)
+  uint64_t wempty[ST];   // one MMA commit
   uint64_t acc_full;
   uint32_t tmem_base;
   int abort_flag;
   unsigned int last;
 };
 
-// Same widening as the large-M kernel: each nibble q lands in the high half of
-// a byte (the signed byte 16*q); both operands share the byte order, the MMA
-// accumulates 256*acc exactly and the epilogue shifts the factor out.
+// Each nibble q of a packed word to the byte 16*q: codes 1,3,5,7 and 0,2,4,6
+// (a signed nibble in the high half of a byte IS the signed byte 16*q).
 __device__ __forceinline__ void widen_word16(uint32_t w, uint32_t& o0, uint32_t& o1) {
   o0 = w & 0xF0F0F0F0u;
   o1 = (w << 4) & 0xF0F0F0F0u;
 }
 
-template <int kUnits>
-__device__ __forceinline__ void widen_tile(const uint8_t* __restrict__ packed, uint8_t* __restrict__ wide, int wt) {
-  constexpr int kPer = (kUnits + kWorkWarps * 32 - 1) / (kWorkWarps * 32);
-#pragma unroll
-  for (int i = 0; i < kPer; ++i) {
-    const int u = wt + i * kWorkWarps * 32;
-    if (kUnits % (kWorkWarps * 32) != 0 && u >= kUnits) break;
-    const int r = u >> 2;
-    const int part = u & 3;
-    const uint4 w = *reinterpret_cast<const uint4*>(packed + u * 16);
-    uint4 c0, c1;
-    widen_word16(w.x, c0.x, c0.y);
-    widen_word16(w.y, c0.z, c0.w);
-    widen_word16(w.z, c1.x, c1.y);
-    widen_word16(w.w, c1.z, c1.w);
-    uint8_t* rowp = wide + (r >> 3) * 1024 + (r & 7) * 128;
-    const int sw = r & 7;
-    *reinterpret_cast<uint4*>(rowp + (((2 * part) ^ sw) << 4)) = c0;
-    *reinterpret_cast<uint4*>(rowp + (((2 * part + 1) ^ sw) << 4)) = c1;
-  }
+// D[tmem] (+)= A[tmem] * B[smem]^T, int8 x int8 -> int32, one CTA.
+__device__ __forceinline__ void mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
 }
+// 32 lanes x 32 consecutive 32-bit columns from registers: thread i of the
+// warp writes row (lane base + i), columns [col, col + 32).
+__device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+      "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+      "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 template <int NP>
 __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[NP]);
@@ -118,6 +137,20 @@ __device__ __forceinline__ void tmem_ld_cols<64>(uint32_t taddr, uint32_t (&r)[6
   tmem_ld_32x32b_x32(taddr + 32, b);
 }
 
+// 32-bit load from the shared memory of CTA `rank` of this cluster, at the
+// offset that `local` (a shared::cta address) has in this CTA.
+__device__ __forceinline__ int32_t ld_shared_cluster_s32(uint32_t local, uint32_t rank) {
+  int32_t v;
+  asm volatile(
+      "{\n\t.reg .b32 ra;\n\t"
+      "mapa.shared::cluster.u32 ra, %1, %2;\n\t"
+      "ld.shared::cluster.s32 %0, [ra];\n\t}"
+      : "=r"(v)
+      : "r"(local), "r"(rank)
+      : "memory");
+  return v;
+}
+
 __device__ __forceinline__ float bf16_to_f(uint16_t b) { return __uint_as_float(static_cast<uint32_t>(b) << 16); }
 __device__ __forceinline__ uint16_t f_to_bf16(float f) {
   const __nv_bfloat16 h = __float2bfloat16_rn(f);
@@ -125,7 +158,7 @@ __device__ __forceinline__ uint16_t f_to_bf16(float f) {
 }
 
 template <int NP, int OUT_S32>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
     smallm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, SmallMArgs args,
                   int kb_per_split, int splits) {
   using Lay = Layout<NP>;
@@ -144,21 +177,34 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nkb = kb1 - kb0;   // >= 1 by construction
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < SP; ++s) {
-      mbar_init(&bars.packed_full[s], 1);
-      mbar_init(&bars.packed_empty[s], kWorkWarps);
+    for (int s = 0; s < Lay::kSP; ++s) {
+      mbar_init(&bars.full[s], 1);
+      mbar_init(&bars.empty[s], kWorkWarps);
     }
-    for (int s = 0; s < SWD; ++s) {
-      mbar_init(&bars.wide_full[s], kWorkWarps);
-      mbar_init(&bars.wide_empty[s], 1);
+    for (int s = 0; s < Lay::kST; ++s) {
+      mbar_init(&bars.wfull[s], kWorkWarps);
+      mbar_init(&bars.wempty[s], 1);
     }
     mbar_init(&bars.acc_full, 1);
     bars.abort_flag = 0;
     fence_mbar_init();
+    tma_prefetch_desc(&tmW);
+    tma_prefetch_desc(&tmX);
   }
   if (warp == 1) {
-    tmem_alloc(&bars.tmem_base, Lay::kTmemCols);
+    tmem_alloc(&bars.tmem_base, kTmemCols);
     tmem_relinquish();
+  }
+  if (!OUT_S32 && warp >= 2) {
+    // epilogue operands, loaded now so that their latency hides behind the stream
+    const int t = threadIdx.x - 64;
+    if (t < WM) {
+      const int64_t n = static_cast<int64_t>(ntile) * WM + t;
+      bars.sw[t] = n < N ? args.sw[n] : 0.0f;
+      bars.bias[t] = (n < N && args.bias != nullptr) ? bf16_to_f(args.bias[n]) : 0.0f;
+    } else if (t < WM + 64) {
+      bars.sx[t - WM] = t - WM < M ? args.sx[t - WM] : 0.0f;
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -167,176 +213,193 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = &bars.abort_flag;
 
   if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       uint32_t ps = 0, ph = 0;
       int issued = 0;
       bool ok = true;
       for (int kb = kb0; kb < kb1; ++kb) {
-        if (!mbar_wait(&bars.packed_empty[ps], ph ^ 1, abort_flag, args.status)) { ok = false; break; }
-        mbar_arrive_expect_tx(&bars.packed_full[ps], Lay::kPackW + Lay::kPackX);
-        tma_load_2d(smem + Lay::kOffPackW + ps * Lay::kPackW, &tmW, &bars.packed_full[ps], kb * BKP, ntile * WM);
-        tma_load_2d(smem + Lay::kOffPackX + ps * Lay::kPackX, &tmX, &bars.packed_full[ps], kb * BKP, 0);
+        if (!mbar_wait(&bars.empty[ps], ph ^ 1, abort_flag, args.status)) { ok = false; break; }
+        mbar_arrive_expect_tx(&bars.full[ps], Lay::kPackW + Lay::kPackX);
+        tma_load_2d(smem + Lay::kOffPackW + ps * Lay::kPackW, &tmW, &bars.full[ps], kb * BKP, ntile * WM);
+        tma_load_2d(smem + Lay::kOffPackX + ps * Lay::kPackX, &tmX, &bars.full[ps], kb * BKP, 0);
         ++issued;
-        if (++ps == SP) { ps = 0; ph ^= 1; }
+        if (++ps == Lay::kSP) { ps = 0; ph ^= 1; }
       }
       if (!ok) {
-        for (int s = 0; s < SP && s < issued; ++s) {
-          const int n_s = issued / SP + (s < issued % SP ? 1 : 0);
-          (void)mbar_wait(&bars.packed_full[s], static_cast<uint32_t>((n_s - 1) & 1), nullptr, nullptr, 100000000ull);
+        for (int s = 0; s < Lay::kSP && s < issued; ++s) {
+          const int n_s = issued / Lay::kSP + (s < issued % Lay::kSP ? 1 : 0);
+          (void)mbar_wait(&bars.full[s], static_cast<uint32_t>((n_s - 1) & 1), nullptr, nullptr, 100000000ull);
         }
       }
     }
   } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_i8(WM, NP);
       uint32_t ws = 0, wph = 0;
-      bool ok = true;
       for (int i = 0; i < nkb; ++i) {
-        if (!mbar_wait(&bars.wide_full[ws], wph, abort_flag, args.status)) { ok = false; break; }
+        if (!mbar_wait(&bars.wfull[ws], wph, abort_flag, args.status)) break;
         tc_fence_after();
-        const uint64_t ad = sw128_kmajor_desc(smem_u32(smem + Lay::kOffWideW + ws * Lay::kWideW));
         const uint64_t bd = sw128_kmajor_desc(smem_u32(smem + Lay::kOffWideX + ws * Lay::kWideX));
+        const uint32_t a_tmem = tmem_base + kTmemA + ws * 32;
 #pragma unroll
         for (int kk = 0; kk < BK / 32; ++kk)
-          mma_i8(tmem_base, ad + 2 * kk, bd + 2 * kk, idesc, (i | kk) != 0 ? 1u : 0u);
-        mma_commit(&bars.wide_empty[ws]);
-        if (++ws == SWD) { ws = 0; wph ^= 1; }
+          mma_i8_ts(tmem_base, a_tmem + kk * 8, bd + 2 * kk, idesc, (i | kk) != 0 ? 1u : 0u);
+        mma_commit(&bars.wempty[ws]);
+        if (++ws == Lay::kST) { ws = 0; wph ^= 1; }
       }
-      (void)ok;
       mma_commit(&bars.acc_full);   // also the drain point on an abort
     }
   } else {
-    const int wt = threadIdx.x - 64;
+    // ------------------------------------------------------------ widen warps
+    // Weights: thread r (= tensor-memory lane) widens weight row r of the
+    // tile, read from the 64-byte-swizzled tile (chunk j of row r at
+    // j ^ ((r >> 1) & 3)), into 32 columns of tensor memory.  Activations:
+    // unit u (16 packed bytes) is part u % 4 of row u / 4; its 32 widened
+    // bytes go to chunks 2 * part and 2 * part + 1 of that row in the
+    // 128-byte-swizzle K-major layout of the B operand.
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
+    const int grp = (warp - 2) / kWorkWarps;
+    const int wt = threadIdx.x - 64 - grp * kWorkWarps * 32;
+    const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + kTmemA;
     uint32_t ps = 0, ph = 0, ws = 0, wph = 0;
     bool ok = true;
-    for (int i = 0; i < nkb; ++i) {
-      if (!warp_wait(&bars.packed_full[ps], ph, abort_flag, args.status) ||
-          !warp_wait(&bars.wide_empty[ws], wph ^ 1, abort_flag, args.status)) { ok = false; break; }
-      widen_tile<WM * BKP / 16>(smem + Lay::kOffPackW + ps * Lay::kPackW, smem + Lay::kOffWideW + ws * Lay::kWideW, wt);
-      widen_tile<NP * BKP / 16>(smem + Lay::kOffPackX + ps * Lay::kPackX, smem + Lay::kOffWideX + ws * Lay::kWideX, wt);
-      fence_async_shared();
+    for (int i = 0; i < nkb; ++i, ps = (ps + 1 == Lay::kSP ? 0 : ps + 1), ph ^= (ps == 0 ? 1u : 0u),
+             ws = (ws + 1 == Lay::kST ? 0 : ws + 1), wph ^= (ws == 0 ? 1u : 0u)) {
+      if (i % kGroups != grp) continue;
+      if (!warp_wait(&bars.full[ps], ph, abort_flag, args.status) ||
+          !warp_wait(&bars.wempty[ws], wph ^ 1, abort_flag, args.status)) { ok = false; break; }
+      {
+        const uint8_t* src = smem + Lay::kOffPackW + ps * Lay::kPackW + r * BKP;
+        const int swz = (r >> 1) & 3;
+        uint32_t v[32];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint4 u = *reinterpret_cast<const uint4*>(src + ((j ^ swz) << 4));
+          widen_word16(u.x, v[8 * j + 0], v[8 * j + 1]);
+          widen_word16(u.y, v[8 * j + 2], v[8 * j + 3]);
+          widen_word16(u.z, v[8 * j + 4], v[8 * j + 5]);
+          widen_word16(u.w, v[8 * j + 6], v[8 * j + 7]);
+        }
+        tmem_st_32x32b_x32(t_lane + ws * 32, v);
+      }
+      {
+        constexpr int kUnits = NP * BKP / 16;
+        const uint8_t* src = smem + Lay::kOffPackX + ps * Lay::kPackX;
+        uint8_t* dst = smem + Lay::kOffWideX + ws * Lay::kWideX;
+#pragma unroll
+        for (int u = wt; u < kUnits; u += kWorkWarps * 32) {
+          const uint4 w = *reinterpret_cast<const uint4*>(src + u * 16);
+          const int rr = u >> 2, part = u & 3;
+          uint4 c0, c1;
+          widen_word16(w.x, c0.x, c0.y);
+          widen_word16(w.y, c0.z, c0.w);
+          widen_word16(w.z, c1.x, c1.y);
+          widen_word16(w.w, c1.z, c1.w);
+          uint8_t* rowp = dst + (rr >> 3) * 1024 + (rr & 7) * 128;
+          *reinterpret_cast<uint4*>(rowp + (((2 * part) ^ (rr & 7)) << 4)) = c0;
+          *reinterpret_cast<uint4*>(rowp + (((2 * part + 1) ^ (rr & 7)) << 4)) = c1;
+        }
+      }
+      tmem_wait_st();
+      fence_async_shared();   // generic-proxy writes, read by the tensor cores
+      tc_fence_before();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(&bars.wide_full[ws]);
-        mbar_arrive(&bars.packed_empty[ps]);
-      }
-      if (++ps == SP) { ps = 0; ph ^= 1; }
-      if (++ws == SWD) { ws = 0; wph ^= 1; }
-    }
-    // ------------------------------------------------------------- epilogue
-    if (ok) (void)warp_wait(&bars.acc_full, 0, abort_flag, args.status);
-    // the four work warps agree before any of them takes the named barriers below
-    asm volatile("bar.sync 1, %0;" ::"r"(kWorkWarps * 32) : "memory");
-    const bool all_ok = *abort_flag == 0;
-    __syncwarp();
-    const int q = warp & 3;
-    const int64_t n = static_cast<int64_t>(ntile) * WM + q * 32 + lane;   // weight row = output column
-    const bool ncol = n < N;
-    uint32_t acc[NP];
-    if (all_ok) {
-      tc_fence_after();
-      tmem_ld_cols<NP>(tmem_base + (static_cast<uint32_t>(q * 32) << 16), acc);
-      tmem_wait_ld();
-#pragma unroll
-      for (int m = 0; m < NP; ++m) acc[m] = static_cast<uint32_t>(static_cast<int32_t>(acc[m]) >> 8);
-    }
-    const int mrows = static_cast<int>(M);
-    bool do_epi = all_ok && splits == 1;
-    if (all_ok && splits > 1) {
-      // this split's partial tile goes to its own slot: no zeroed memory needed
-      if (ncol) {
-        int32_t* slot = args.partial + static_cast<int64_t>(split) * M * N;
-#pragma unroll
-        for (int m = 0; m < NP; ++m)
-          if (m < mrows) __stcg(slot + static_cast<int64_t>(m) * N + n, static_cast<int>(acc[m]));
-      }
-      __threadfence();
-      asm volatile("bar.sync 1, %0;" ::"r"(kWorkWarps * 32) : "memory");
-      if (wt == 0) {
-        // wraps back to 0 on the last arrival, leaving the counter ready for the next call
-        const unsigned int old = atomicInc(args.counters + ntile, static_cast<unsigned int>(splits - 1));
-        bars.last = (old == static_cast<unsigned int>(splits - 1)) ? 1u : 0u;
-      }
-      asm volatile("bar.sync 1, %0;" ::"r"(kWorkWarps * 32) : "memory");
-      if (bars.last) {
-        __threadfence();
-        if (ncol) {
-          // sum the slots in split order (integer addition: exact)
-#pragma unroll
-          for (int m = 0; m < NP; ++m) {
-            if (m < mrows) {
-              int sum = 0;
-              for (int sp = 0; sp < splits; ++sp)
-                sum += __ldcg(args.partial + (static_cast<int64_t>(sp) * M + m) * N + n);
-              acc[m] = static_cast<uint32_t>(sum);
-            }
-          }
-        }
-        do_epi = true;
+        mbar_arrive(&bars.wfull[ws]);
+        mbar_arrive(&bars.empty[ps]);
       }
     }
-    if (do_epi && ncol) {
-      if (OUT_S32) {
-        int32_t* out = reinterpret_cast<int32_t*>(args.out);
+    // The first group moves this CTA's partial tile from tensor memory to
+    // shared memory (the packed-weight ring, idle once the accumulator is
+    // complete), laid out part[m][r] so that a warp's rows are contiguous.
+    if (grp == 0) {
+      if (ok) (void)warp_wait(&bars.acc_full, 0, abort_flag, args.status);
+      if (*abort_flag == 0) {
+        tc_fence_after();
+        uint32_t acc[NP];
+        tmem_ld_cols<NP>(tmem_base + (static_cast<uint32_t>(q * 32) << 16), acc);
+        tmem_wait_ld();
+        int32_t* part = reinterpret_cast<int32_t*>(smem + Lay::kOffPackW);
 #pragma unroll
-        for (int m = 0; m < NP; ++m)
-          if (m < mrows) out[static_cast<int64_t>(m) * args.ldo + n] = static_cast<int32_t>(acc[m]);
-      } else {
-        uint16_t* out = reinterpret_cast<uint16_t*>(args.out);
-        const float swn = args.sw[n];
-        const float bn = args.bias != nullptr ? bf16_to_f(args.bias[n]) : 0.0f;
-#pragma unroll
-        for (int m = 0; m < NP; ++m) {
-          if (m < mrows) {
-            float y = __fmul_rn(__fmul_rn(__int2float_rn(static_cast<int>(acc[m])), args.sx[m]), swn);
-            if (args.bias != nullptr) y = __fadd_rn(y, bn);
-            out[static_cast<int64_t>(m) * args.ldo + n] = f_to_bf16(y);
-          }
-        }
+        for (int m = 0; m < NP; ++m) part[m * WM + r] = static_cast<int32_t>(acc[m]) >> 8;
       }
     }
   }
 
+  // ---- K-slice reduction across the cluster (one cluster per weight tile,
+  // one CTA per K slice), through distributed shared memory: CTA c sums rows
+  // [c*R, c*R + R) of the tile over the cluster's partials in rank order
+  // (integer addition: exact and deterministic), applies the epilogue and
+  // writes those outputs.
   tc_fence_before();
   __syncthreads();
+  cluster_sync();   // every CTA's partial tile is in its shared memory
+  {
+    const int R = (WM + splits - 1) / splits;
+    const int r0 = split * R;
+    const int rows = min(WM - r0, R);
+    const int mrows = static_cast<int>(M);
+    const uint32_t part_local = smem_u32(smem + Lay::kOffPackW);
+    for (int idx = threadIdx.x; idx < rows * mrows; idx += kThreads) {
+      const int m = idx / rows;
+      const int rr = r0 + (idx - m * rows);
+      const int64_t n = static_cast<int64_t>(ntile) * WM + rr;   // weight row = output column
+      if (n >= N) continue;
+      const uint32_t off = static_cast<uint32_t>(m * WM + rr) * 4u;
+      int32_t sum = 0;
+      for (int c = 0; c < splits; ++c) sum += ld_shared_cluster_s32(part_local + off, static_cast<uint32_t>(c));
+      if (OUT_S32) {
+        reinterpret_cast<int32_t*>(args.out)[static_cast<int64_t>(m) * args.ldo + n] = sum;
+      } else {
+        float y = __fmul_rn(__fmul_rn(__int2float_rn(sum), bars.sx[m]), bars.sw[rr]);
+        if (args.bias != nullptr) y = __fadd_rn(y, bars.bias[rr]);
+        reinterpret_cast<uint16_t*>(args.out)[static_cast<int64_t>(m) * args.ldo + n] = f_to_bf16(y);
+      }
+    }
+  }
+  cluster_sync();   // no CTA leaves while its partial tile may still be read
   if (warp == 1) {
     // the MMA thread's final commit arrives when every MMA has completed
     if (lane == 0) (void)mbar_wait(&bars.acc_full, 0, nullptr, nullptr, 100000000ull);
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, Lay::kTmemCols);
+    tmem_dealloc(tmem_base, kTmemCols);
   }
 }
 
-template <int NP>
-cudaError_t launch_np(const CUtensorMap& tmW, const CUtensorMap& tmX, const SmallMArgs& a, int kb_per, int splits,
-                      int ntiles, cudaStream_t stream) {
-  using Lay = Layout<NP>;
-  const int grid = ntiles * splits;
-  cudaError_t e;
-  if (a.out_s32) {
-    e = cudaFuncSetAttribute(smallm_kernel<NP, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kAlloc);
-    if (e != cudaSuccess) return e;
-    smallm_kernel<NP, 1><<<grid, kThreads, Lay::kAlloc, stream>>>(tmW, tmX, a, kb_per, splits);
-  } else {
-    e = cudaFuncSetAttribute(smallm_kernel<NP, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kAlloc);
-    if (e != cudaSuccess) return e;
-    smallm_kernel<NP, 0><<<grid, kThreads, Lay::kAlloc, stream>>>(tmW, tmX, a, kb_per, splits);
-  }
-  return cudaGetLastError();
+constexpr int kMaxSplits = 8;   // the portable cluster size
+
+template <int NP, int OUT_S32>
+void fill_cfg(cudaLaunchConfig_t* cfg, cudaLaunchAttribute* attr, int ctas, int splits, cudaStream_t stream) {
+  *cfg = cudaLaunchConfig_t{};
+  cfg->gridDim = dim3(static_cast<unsigned>(ctas), 1, 1);
+  cfg->blockDim = dim3(kThreads, 1, 1);
+  cfg->dynamicSmemBytes = Layout<NP>::kAlloc;
+  cfg->stream = stream;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(splits);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg->attrs = attr;
+  cfg->numAttrs = 1;
 }
 
-}  // namespace
-
-// Split plan shared by the launcher and the workspace query.  It is sized for
-// the 148 SMs of a B200 (about two CTAs per SM) rather than the device's own
-// count, so that the workspace size stays a pure function of the shape.
-constexpr int kPlanSms = 148;
-static void smallm_plan(int64_t N, int64_t K, int num_sms, int* ntiles, int* kb_per, int* splits) {
+// Split plan: K slices per 128-row weight tile.  Two CTAs fit on an SM
+// (registers, shared memory and tensor memory each allow two), and clusters
+// pack into the GPCs with some loss, so the plan keeps the grid within 85% of
+// 2 x 148 CTAs -- every cluster is then resident at once (a second wave of a
+// few clusters would double the kernel's time) -- with at most kMaxSplits
+// slices and at least one k-block per slice.
+void smallm_plan(int64_t N, int64_t K, int* ntiles, int* kb_per, int* splits) {
+  constexpr int kMaxCtas = static_cast<int>(0.85 * 2 * 148);
   const int nt = static_cast<int>((N + WM - 1) / WM);
   const int num_kb = static_cast<int>((K + BK - 1) / BK);
-  int s = static_cast<int>((2.0 * num_sms) / nt + 0.5);
+  int s = kMaxCtas / nt;
   if (s < 1) s = 1;
+  if (s > kMaxSplits) s = kMaxSplits;
   if (s > num_kb) s = num_kb;
   const int per = (num_kb + s - 1) / s;
   *ntiles = nt;
@@ -344,21 +407,44 @@ static void smallm_plan(int64_t N, int64_t K, int num_sms, int* ntiles, int* kb_
   *splits = (num_kb + per - 1) / per;
 }
 
-size_t smallm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+template <int NP, int OUT_S32>
+cudaError_t launch_cfg(const CUtensorMap& tmW, const CUtensorMap& tmX, const SmallMArgs& a, cudaStream_t stream) {
+  using Lay = Layout<NP>;
+  static bool attrs_set[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!attrs_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(smallm_kernel<NP, OUT_S32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Lay::kAlloc);
+    if (e != cudaSuccess) return e;
+    // the whole unified L1/shared array as shared memory, so that two CTAs fit per SM
+    e = cudaFuncSetAttribute(smallm_kernel<NP, OUT_S32>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    attrs_set[dev] = true;
+  }
   int nt, per, splits;
-  smallm_plan(N, K, kPlanSms, &nt, &per, &splits);
-  size_t part = splits > 1 ? static_cast<size_t>(splits) * M * N * 4 : 0;
-  return kSmallMCounterBytes + (part + 255) / 256 * 256;
+  smallm_plan(a.N, a.K, &nt, &per, &splits);
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute attr[1];
+  fill_cfg<NP, OUT_S32>(&cfg, attr, nt * splits, splits, stream);
+  return cudaLaunchKernelEx(&cfg, smallm_kernel<NP, OUT_S32>, tmW, tmX, a, per, splits);
 }
 
-cudaError_t smallm_launch_tm(const CUtensorMap& tmW, const CUtensorMap& tmX, const SmallMArgs& a, int num_sms,
+template <int NP>
+cudaError_t launch_np(const CUtensorMap& tmW, const CUtensorMap& tmX, const SmallMArgs& a, cudaStream_t stream) {
+  cudaError_t e = a.out_s32 ? launch_cfg<NP, 1>(tmW, tmX, a, stream) : launch_cfg<NP, 0>(tmW, tmX, a, stream);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t smallm_launch_tm(const CUtensorMap& tmW, const CUtensorMap& tmX, const SmallMArgs& a,
                              cudaStream_t stream) {
-  (void)num_sms;
-  int nt, per, splits;
-  smallm_plan(a.N, a.K, kPlanSms, &nt, &per, &splits);
-  if (a.M <= 16) return launch_np<16>(tmW, tmX, a, per, splits, nt, stream);
-  if (a.M <= 32) return launch_np<32>(tmW, tmX, a, per, splits, nt, stream);
-  return launch_np<64>(tmW, tmX, a, per, splits, nt, stream);
+  if (a.M <= 16) return launch_np<16>(tmW, tmX, a, stream);
+  if (a.M <= 32) return launch_np<32>(tmW, tmX, a, stream);
+  return launch_np<64>(tmW, tmX, a, stream);
 }
 
 int smallm_rows_padded(int64_t M) { return M <= 16 ? 16 : (M <= 32 ? 32 : 64); }
@@ -366,47 +452,11 @@ int smallm_rows_padded(int64_t M) { return M <= 16 ? 16 : (M <= 32 ? 32 : 64); }
 }  // namespace w4a4
 
 // ---------------------------------------------------------------------------
-// Small-M linear that allocates nothing (w4a4_linear_noalloc in w4a4.h).
-//
-// Same kernel and launch as the workspace-taking path; only the scratch is
-// different: the arrival counters and split-K slots live in a fixed array of
-// this library's own device memory instead of a caller workspace.
+// Small-M linear that allocates nothing (w4a4_linear_noalloc in w4a4.h): the
+// small-M kernel reduces its K slices on chip, so it needs no scratch memory
+// at all; this entry takes no workspace argument.
 // ---------------------------------------------------------------------------
-#include <mutex>
-
 #include "w4a4.h"
-
-namespace {
-
-constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;   // 4 MiB: counter block + split-K slots
-static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
-
-constexpr int kNoAllocMaxDevices = 64;
-void* g_noalloc_ptr[kNoAllocMaxDevices] = {nullptr};   // device address of the array, per device
-std::mutex g_noalloc_mu;
-
-// Device address of the scratch array on the current device.  The host-side
-// name g_noalloc_scratch is only a stand-in for the symbol, never a device
-// pointer, so its address is resolved once per device with
-// cudaGetSymbolAddress (with that device current) and cached; the same first
-// call clears the counter block on `stream` (the counters must start at zero;
-// every completed call leaves them at zero again).
-int noalloc_scratch(uint8_t** out, cudaStream_t stream) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return W4A4_ERR_CUDA;
-  if (dev < 0 || dev >= kNoAllocMaxDevices) return W4A4_ERR_DEVICE;
-  std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return W4A4_ERR_CUDA;
-    if (cudaMemsetAsync(p, 0, w4a4::kSmallMCounterBytes, stream) != cudaSuccess) return W4A4_ERR_CUDA;
-    g_noalloc_ptr[dev] = p;
-  }
-  *out = static_cast<uint8_t*>(g_noalloc_ptr[dev]);
-  return W4A4_OK;
-}
-
-}  // namespace
 
 extern "C" int w4a4_linear_noalloc(const int8_t* Xq, const float* sx, const int8_t* Wq, const float* sw,
                                    const uint16_t* bias, uint16_t* y, int64_t M, int64_t N, int64_t K, int64_t ldy,
@@ -414,15 +464,11 @@ extern "C" int w4a4_linear_noalloc(const int8_t* Xq, const float* sx, const int8
   using namespace w4a4;
   int st = validate_linear(Xq, sx, Wq, sw, bias, y, M, N, K, ldy, 0);
   if (st != W4A4_OK) return st;
-  if (M < 1 || M > kSmallMMax || N > kSmallMMaxN) return W4A4_ERR_SHAPE;
-  if (smallm_workspace_bytes(M, N, K) > kNoAllocScratchBytes) return W4A4_ERR_WORKSPACE;
+  if (M < 1 || M > kSmallMMax) return W4A4_ERR_SHAPE;
   DeviceInfo* dev = nullptr;
   if ((st = current_device(&dev)) != W4A4_OK) return st;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  uint8_t* scratch = nullptr;
-  if ((st = noalloc_scratch(&scratch, s)) != W4A4_OK) return st;
   CUtensorMap tmW, tmX;
-  if ((st = packed_map(&tmW, Wq, N, K, WM)) != W4A4_OK) return st;
+  if ((st = packed_map(&tmW, Wq, N, K, WM, true)) != W4A4_OK) return st;
   if ((st = packed_map(&tmX, Xq, M, K, smallm_rows_padded(M))) != W4A4_OK) return st;
   SmallMArgs a{};
   a.xq = Xq;
@@ -436,8 +482,6 @@ extern "C" int w4a4_linear_noalloc(const int8_t* Xq, const float* sx, const int8
   a.out = y;
   a.ldo = ldy;
   a.out_s32 = 0;
-  a.counters = reinterpret_cast<unsigned int*>(scratch);
-  a.partial = reinterpret_cast<int32_t*>(scratch + kSmallMCounterBytes);
   a.status = dev->status;
-  return smallm_launch_tm(tmW, tmX, a, dev->num_sms, s) == cudaSuccess ? W4A4_OK : W4A4_ERR_CUDA;
+  return smallm_launch_tm(tmW, tmX, a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? W4A4_OK : W4A4_ERR_CUDA;
 }

@@ -17,8 +17,9 @@ struct DeviceInfo {
 };
 // The current device (must be sm_100); W4A4_OK or an error status.
 int current_device(DeviceInfo** out);
-// TMA map over a packed int4 matrix [rows, K/2] bytes with box {64, box_rows}.
-int packed_map(CUtensorMap* map, const int8_t* base, int64_t rows, int64_t K, int box_rows);
+// TMA map over a packed int4 matrix [rows, K/2] bytes with box {64, box_rows}
+// (64-byte swizzle in shared memory when swizzle64).
+int packed_map(CUtensorMap* map, const int8_t* base, int64_t rows, int64_t K, int box_rows, bool swizzle64 = false);
 // Argument checks of w4a4_linear (out_s32 = 0) / w4a4_gemm_s32 (out_s32 = 1).
 int validate_linear(const int8_t* Xq, const float* sx, const int8_t* Wq, const float* sw, const uint16_t* bias,
                     const void* y, int64_t M, int64_t N, int64_t K, int64_t ldy, int out_s32);
@@ -65,21 +66,15 @@ struct SmallMArgs {
   void* out;
   int64_t ldo;
   int out_s32;
-  int32_t* partial;       // workspace: [splits, M, N] int32 split-K partial tiles
-  unsigned int* counters; // workspace: one arrival counter per N tile (zero between calls)
   unsigned int* status;   // device status word
 };
-// tmW: packed weights [N, K/2] bytes, box {64, 128}; tmX: packed activations
-// [M, K/2] bytes, box {64, smallm_rows_padded(M)}.
-cudaError_t smallm_launch_tm(const CUtensorMap& tmW, const CUtensorMap& tmX, const SmallMArgs& a, int num_sms,
+// tmW: packed weights [N, K/2] bytes, box {64, 128}, 64-byte swizzle; tmX:
+// packed activations [M, K/2] bytes, box {64, smallm_rows_padded(M)}.
+// Launched as clusters of up to 8 CTAs (one cluster per 128-row weight tile,
+// one CTA per K slice); needs no workspace.
+cudaError_t smallm_launch_tm(const CUtensorMap& tmW, const CUtensorMap& tmX, const SmallMArgs& a,
                              cudaStream_t stream);
 int smallm_rows_padded(int64_t M);
-size_t smallm_workspace_bytes(int64_t M, int64_t N, int64_t K);
 constexpr int kSmallMMax = 64;
-// Every workspace starts with a block of arrival counters (one per 128-row
-// weight tile, so N <= 8192 * 128) that must be zero before the first call
-// and is left zero by every call.
-constexpr size_t kSmallMCounterBytes = 32768;
-constexpr int64_t kSmallMMaxN = static_cast<int64_t>(kSmallMCounterBytes / 4) * 128;
 
 }  // namespace w4a4
