@@ -62,10 +62,14 @@ constexpr int SWD = 4;          // widened ring depth
 // Warp roles.  A warp runs on SM sub-partition (warp % 4).  The threads that
 // issue tcgen05.mma and TMA instructions hold their sub-partition's issue
 // slot for long stretches, so they share sub-partition 0 with one epilogue
-// warp and no widen warp; the nine widen warps sit three to a sub-partition on
-// 1..3, next to one epilogue warp each (an epilogue warp may only read the
-// tensor-memory lane quarter warp % 4).
-constexpr int kWidenWarps = 9;
+// warp and no widen warp; the widen warps sit on sub-partitions 1..3 (nine
+// slots: warps 1-3, 5-7, 9-11), next to one epilogue warp each (an epilogue
+// warp may only read the tensor-memory lane quarter warp % 4).
+// The widen warps can form kWGroups groups that take turns by k-block; with
+// the shared-memory bandwidth as the limit, one group of eight warps (four
+// 16-byte units per thread, the ninth slot idle) measured fastest.
+constexpr int kWGroups = 1;
+constexpr int kWidenWarps = 8;   // per group
 constexpr int kEpiWarps = 4;
 constexpr int kWarpMma = 0;
 constexpr int kWarpTma = 4;
@@ -74,6 +78,7 @@ __device__ __forceinline__ bool is_epi_warp(int w) { return w == 8 || w >= 13; }
 __device__ __forceinline__ bool is_widen_warp(int w) { return w != 0 && w != 4 && w != 8 && w < 12; }
 // widen warps 1,2,3,5,6,7,9,10,11 -> 0..8
 __device__ __forceinline__ int widen_index(int w) { return w - 1 - (w > 4) - (w > 8); }
+static_assert(kWGroups * kWidenWarps <= 9, "nine widen warp slots");
 constexpr int kTmemCols = 2 * BN;   // two int32 accumulators of BN columns
 
 constexpr uint32_t kWideA = HM * BK;     // 16 KB
@@ -214,6 +219,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   cluster_sync();   // barriers and tensor memory of both CTAs are ready
   tc_fence_after();
+  // launched with programmatic stream serialization: the set-up above may
+  // overlap the previous kernel (the activation quantiser of a fused layer);
+  // its outputs are read only after this point
+  griddep_wait();
   const uint32_t tmem_base = bars.tmem_base;
   volatile int* abort_flag = &bars.abort_flag;
 
@@ -297,11 +306,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (is_widen_warp(warp)) {
     // ------------------------------------------------------------ widen warps
-    const int wt = widen_index(warp) * 32 + lane;
+    const int grp = widen_index(warp) / kWidenWarps;
+    const int wt = (widen_index(warp) % kWidenWarps) * 32 + lane;
     uint32_t ps = 0, ph = 0, ws = 0, wph = 0;
-    bool ok = true;
+    uint32_t gk = 0;
+    bool ok = grp < kWGroups;   // spare warp slots stay idle
     for (int t = cluster; t < tiles && ok; t += nclusters) {
-      for (int kb = 0; kb < num_kb; ++kb) {
+      for (int kb = 0; kb < num_kb; ++kb, ++gk) {
+        if (static_cast<int>(gk % kWGroups) != grp) {
+          if (++ps == SP) { ps = 0; ph ^= 1; }
+          if (++ws == SWD) { ws = 0; wph ^= 1; }
+          continue;
+        }
         if (!warp_wait(&bars.packed_full[ps], ph, abort_flag, args.status) ||
             !warp_wait_cluster(&bars.wide_empty[ws], wph ^ 1, abort_flag, args.status)) { ok = false; break; }
         widen_units(smem + kOffPack + ps * kPStage, smem + ws * kStage, wt);
@@ -475,13 +491,15 @@ cudaError_t launch(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtenso
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = kSmemAlloc;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<OUT_S32>, tmA, tmB, tmY, a);
 }
 

@@ -178,6 +178,10 @@ __global__ void __maxnreg__(96)
   const size_t row_bytes = static_cast<size_t>(K) * sizeof(TIn);
   const size_t stage_bytes = static_cast<size_t>(P) * row_bytes;
 
+  // every CTA of this persistent grid is resident now: the next kernel of the
+  // stream (the GEMM of a fused layer) may be scheduled as SMs free up; it
+  // waits for this grid's writes before it reads them
+  griddep_launch_dependents();
   for (int i = tid; i < 3 * kMaxRows; i += blockDim.x) (&row_amax[0][0])[i] = 0u;
   if (tid == 0) {
     for (int i = 0; i < kMaxStages; ++i) mbar_init(&full[i], 1);

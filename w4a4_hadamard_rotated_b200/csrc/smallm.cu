@@ -195,6 +195,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     tmem_alloc(&bars.tmem_base, kTmemCols);
     tmem_relinquish();
   }
+  // launched with programmatic stream serialization: the set-up above may
+  // overlap the previous kernel (the activation quantiser of a fused layer);
+  // its outputs are read only after this point
+  griddep_wait();
   if (!OUT_S32 && warp >= 2) {
     // epilogue operands, loaded now so that their latency hides behind the stream
     const int t = threadIdx.x - 64;
@@ -426,8 +430,11 @@ cudaError_t launch_cfg(const CUtensorMap& tmW, const CUtensorMap& tmX, const Sma
   int nt, per, splits;
   smallm_plan(a.N, a.K, &nt, &per, &splits);
   cudaLaunchConfig_t cfg;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   fill_cfg<NP, OUT_S32>(&cfg, attr, nt * splits, splits, stream);
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, smallm_kernel<NP, OUT_S32>, tmW, tmX, a, per, splits);
 }
 
