@@ -32,7 +32,10 @@ N_SETS = 5
 # DRAM bytes (read + write) per launch from ncu captures of the current
 # kernels, keyed by (kernel, workload); a kernel that changed since its
 # capture has no entry (traffic reported as null).  Figures: profiles/.
-MEASURED_TRAFFIC = {}
+MEASURED_TRAFFIC = {
+    ("gemm_tc", "square"): 11.90e6 + 0.05e6,                 # profiles/gemm_tc_square_4608x3072x3072.md
+    ("smallm", "smallm_16_12288_3072"): 18.98e6 + 0.0,      # profiles/smallm_16x3072x12288.md
+}
 
 
 def load_peaks():
