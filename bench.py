@@ -196,9 +196,10 @@ def run_reference(args, cfg, world, rank):
 
 
 def workload_from_name(name):
-    """square (default, the headline layer), mlp_up, mlp_down, or
+    """square (default, the headline layer), mlp_up, mlp_down,
     smallm_M_N_K (decode-like, e.g. smallm_16_12288_3072 = 16 rows, N=12288,
-    K=3072)."""
+    K=3072), or stack_gG (the 60-linear transformer block stack at M=32760
+    with group size G; handled by run_stack)."""
     if name == "square":
         return workloads.SQUARE
     if name == "mlp_up":
@@ -428,6 +429,92 @@ def run_impl(args, cfg, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+def run_stack(args, g, world, rank):
+    """The transformer-block linear stack at M = 32760 (10 blocks of q, k, v,
+    out 5120x5120 and an MLP 5120->13824->5120): per block one quantised
+    activation feeds q, k and v (quantise once, three GEMMs); out reads v's
+    output, up reads out's, and down reads GELU(up) (GELU inside the
+    quantiser).  A step is the whole 60-linear stack.  Weights are drawn on
+    the GPU from a seeded generator, rotated and quantised once; inputs are
+    synthetic like the other workloads.  Every activation (335 MB and more)
+    exceeds L2, so every layer reads its operands cold."""
+    import w4a4_hadamard_rotated_b200 as w4
+    w4.load_library()
+    device = torch.device("cuda", torch.cuda.current_device())
+    layers = workloads.block_stack(g=g)
+    M = layers[0].M
+    gen = torch.Generator(device=device).manual_seed(1234 + g)
+    weights = []
+    for cfg in layers:
+        W = torch.randn(cfg.N, cfg.K, generator=gen, device=device) * 0.02
+        b = (torch.randn(cfg.N, generator=gen, device=device) * 0.01).to(torch.bfloat16)
+        Wq, sw = w4.quantize_weight(W, g)
+        del W
+        weights.append((Wq, sw, b))
+    x0 = workloads.make_activation(M, 5120, seed=7, outlier_frac=0.005, outlier_scale=30.0).to(device)
+    Xq = torch.empty(M, 5120 // 2, dtype=torch.int8, device=device)
+    sx = torch.empty(M, dtype=torch.float32, device=device)
+    qkv = [torch.empty(M, 5120, dtype=torch.bfloat16, device=device) for _ in range(3)]
+    h_out = torch.empty(M, 5120, dtype=torch.bfloat16, device=device)
+    h_up = torch.empty(M, 13824, dtype=torch.bfloat16, device=device)
+    h_down = torch.empty(M, 5120, dtype=torch.bfloat16, device=device)
+
+    def step(i):
+        x = x0
+        for blk in range(len(layers) // 6):
+            wq = weights[6 * blk: 6 * blk + 6]
+            w4.quantize_activation(x, g, 0, out=(Xq, sx))
+            for j in range(3):
+                w4.linear(Xq, sx, wq[j][0], wq[j][1], wq[j][2], out=qkv[j])
+            w4.linear_fused(qkv[2], wq[3][0], wq[3][1], wq[3][2], g, 0, out=h_out)
+            w4.linear_fused(h_out, wq[4][0], wq[4][1], wq[4][2], g, 0, out=h_up)
+            w4.linear_fused(h_up, wq[5][0], wq[5][1], wq[5][2], g, 1, out=h_down)
+            x = h_down
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    loop = GraphLoop(step, args.steps)
+    loop.run()
+    sampler = ClockSampler(device.index) if rank == 0 else None
+    if sampler:
+        sampler.start()
+    torch.cuda.synchronize()
+    barrier(world)
+    dt = time_graph(loop)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop() if sampler else None
+    dt_max = max_over_ranks(dt, world)
+    del loop
+    if not torch.isfinite(h_down.float()).all():
+        raise RuntimeError("the stack produced non-finite values")
+    err = w4.last_device_error()
+    if err != 0:
+        raise RuntimeError(f"device status {err} after the benchmark")
+    if rank != 0:
+        return
+    ops = float(sum(c.ops() for c in layers))
+    ms = dt_max / args.steps * 1e3
+    peaks, kind = load_peaks()
+    int8_peak = peaks.get("bf16_tflops", FALLBACK["bf16_tflops"]) * INT8_OVER_BF16
+    line = {
+        "metric": "W4A4 linear TOPS (fused quant+GEMM), transformer block stack at M=32760",
+        "value": world * ops * args.steps / dt_max / 1e12, "unit": "TOPS", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "s4xs4->s32", "data": "synthetic",
+        "config": {"workload": f"block stack 10 x (q,k,v,out 5120^2; up 5120->13824; down 13824->5120) M={M} g{g}",
+                   "linears_per_step": len(layers), "qkv_share_one_quantised_activation": True,
+                   "l2": "every activation exceeds L2", "launch": "CUDA graphs of the stack, replayed",
+                   "parallelism": f"replicas x{world}"},
+        "us_per_linear": ms * 1e3 / len(layers),
+        "tensor_fraction": ops / (dt_max / args.steps) / 1e12 / int8_peak,
+        "gpu_launches": 17 * (len(layers) // 6) * args.steps,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -435,11 +522,25 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="square",
-                    help="square (default: 4608x3072->3072), mlp_up, mlp_down, or smallm_M_N_K")
+                    help="square (default: 4608x3072->3072), mlp_up, mlp_down, smallm_M_N_K, or stack_gG "
+                         "(the 60-linear block stack at M=32760, group size G in 64/128/256)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     world, rank, local = dist_setup()
+    if args.workload.startswith("stack_g"):
+        g = int(args.workload[len("stack_g"):])
+        try:
+            if args.impl == "reference":
+                print(json.dumps({"impl": "reference", "unavailable": "the stack workload has no CPU-oracle arm "
+                                  "(60 layers at M=32760); use the single-layer workloads"}), flush=True)
+            else:
+                run_stack(args, g, world, rank)
+        finally:
+            if world > 1:
+                import torch.distributed as dist
+                dist.destroy_process_group()
+        return
     cfg = workload_from_name(args.workload)
     try:
         if args.impl == "reference":

@@ -301,3 +301,31 @@ def test_quantize_exact_ties_follow_round_half_even(cuda_lib):
     assert np.array_equal(Xq.cpu().numpy(), ref["packed"])
     assert np.array_equal(sx.cpu().numpy(), ref["scale"])
     assert np.sum(orc.boundary_window(ref["v"], 0.0)) > 1000   # the ties are really there
+
+
+def test_block_stack_chain_one_quantised_activation(cuda_lib):
+    """One transformer block of the stack workload at reduced width: q, k and
+    v read one quantised activation (identical to three fused calls), out
+    reads v's output, up reads out's, down reads GELU(up); every layer of the
+    chain matches the oracle on its GPU input."""
+    M, D, F, g = 300, 1024, 2816, 128
+    x = workloads.make_activation(M, D, seed=21, outlier_frac=0.005, outlier_scale=30.0)
+    shapes = {"q": (D, D), "k": (D, D), "v": (D, D), "out": (D, D), "up": (D, F), "down": (F, D)}
+    Ws = {nm: workloads.make_weight(N, K, seed=30 + i) for i, (nm, (K, N)) in enumerate(shapes.items())}
+    bs = {nm: workloads.make_bias(N, seed=40 + i) for i, (nm, (K, N)) in enumerate(shapes.items())}
+    Wq = {nm: cuda_lib.quantize_weight(W.cuda(), g) for nm, W in Ws.items()}
+    xc = x.cuda()
+    Xq, sx = cuda_lib.quantize_activation(xc, g)
+    qkv = {}
+    for nm in ("q", "k", "v"):
+        qkv[nm] = cuda_lib.linear(Xq, sx, Wq[nm][0], Wq[nm][1], bs[nm].cuda())
+        fused = cuda_lib.linear_fused(xc, Wq[nm][0], Wq[nm][1], bs[nm].cuda(), g)
+        assert torch.equal(qkv[nm].view(torch.int16), fused.view(torch.int16))
+    rows = _sample_rows(M, 24, seed=5)
+    cfg = lambda nm, act=0: workloads.Linear(f"stack {nm}", M=M, K=shapes[nm][0], N=shapes[nm][1], g=g, act=act)
+    for nm in ("q", "k", "v"):
+        _check_layer(cuda_lib, cfg(nm), x, Ws[nm], bs[nm], rows=rows, y=qkv[nm])
+    y_out = _check_layer(cuda_lib, cfg("out"), qkv["v"].cpu(), Ws["out"], bs["out"], rows=rows)
+    y_up = _check_layer(cuda_lib, cfg("up"), y_out.cpu(), Ws["up"], bs["up"], rows=rows)
+    y_down = _check_layer(cuda_lib, cfg("down", act=1), y_up.cpu(), Ws["down"], bs["down"], rows=rows)
+    assert torch.isfinite(y_down.float()).all()
