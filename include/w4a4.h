@@ -124,7 +124,9 @@ size_t w4a4_fused_workspace_bytes(int64_t M, int64_t N, int64_t K);
 /*
  * Raw int32 accumulators acc[m, n] = sum_k qx[m,k] * qw[n,k] (no epilogue),
  * for bit-exact checks of the GEMM.  path: 0 = tcgen05 tensor-core kernel,
- * 1 = small-M weight-streaming kernel (M <= 64 only).
+ * 1 = small-M weight-streaming kernel (M <= 64 only), 2 = a comparison
+ * kernel in the pages' own design (warp-level mma.m16n8k64.s4 fed from
+ * shared memory), kept to measure the tcgen05 kernel against.
  *   acc [M, N] int32 output with row stride ldc >= N, ldc % 4 == 0.
  * Other rules as for w4a4_linear.
  */

@@ -98,7 +98,7 @@ def test_fused_rejects_bad_arguments(lib):
 
 def test_gemm_s32_rejects_bad_arguments(lib):
     f = lib.w4a4_gemm_s32
-    assert f(FAKE, FAKE, FAKE, 128, 256, 256, 256, 2, NULL, 0, NULL) == 9      # path
+    assert f(FAKE, FAKE, FAKE, 128, 256, 256, 256, 3, NULL, 0, NULL) == 9      # path
     assert f(FAKE, FAKE, FAKE, 65, 256, 256, 256, 1, NULL, 0, NULL) == 2       # small-M path, M > 64
     assert f(FAKE, FAKE, FAKE, 16, 256, 256, 254, 0, NULL, 0, NULL) == 2       # ldc < N
 

@@ -329,3 +329,12 @@ def test_block_stack_chain_one_quantised_activation(cuda_lib):
     y_up = _check_layer(cuda_lib, cfg("up"), y_out.cpu(), Ws["up"], bs["up"], rows=rows)
     y_down = _check_layer(cuda_lib, cfg("down", act=1), y_up.cpu(), Ws["down"], bs["down"], rows=rows)
     assert torch.isfinite(y_down.float()).all()
+
+
+@pytest.mark.parametrize("M,N,K", [(300, 392, 416), (128, 256, 128), (129, 520, 3072), (65, 8, 32), (1000, 1032, 640)])
+def test_gemm_legacy_mma_sync_exact(cuda_lib, M, N, K):
+    """The warp-level mma.m16n8k64.s4 comparison kernel gives the same int32
+    accumulators as the oracle."""
+    qa, qb = _codes((M, K), 51 + M), _codes((N, K), 52 + N)
+    acc = cuda_lib.gemm_s32(_packed_cuda(qa), _packed_cuda(qb), path=2).cpu().numpy()
+    assert np.array_equal(acc, orc.gemm_s32(orc.pack_int4(qa), orc.pack_int4(qb)))

@@ -178,7 +178,8 @@ def linear_fused(x, Wq, sw, bias=None, g=128, act=0, out=None):
 
 
 def gemm_s32(Xq, Wq, path=0, out=None):
-    """Raw int32 accumulators acc [M, N] (path 0: tcgen05 kernel, 1: small-M kernel)."""
+    """Raw int32 accumulators acc [M, N] (path 0: tcgen05 kernel, 1: small-M
+    kernel, 2: the warp-level mma.sync comparison kernel)."""
     lib = load_library()
     _need_cuda(Xq, torch.int8, "Xq")
     _need_cuda(Wq, torch.int8, "Wq")

@@ -142,13 +142,22 @@ int check_gemm_shape(int64_t M, int64_t N, int64_t K) {
 
 
 // Shared body of w4a4_linear / w4a4_gemm_s32 after validation.  path 0: the
-// tcgen05 tensor-core kernel; 1: the small-M weight-streaming kernel.
+// tcgen05 tensor-core kernel; 1: the small-M weight-streaming kernel; 2: the
+// warp-level mma.sync comparison kernel (int32 output only).
 int run_linear(const int8_t* Xq, const float* sx, const int8_t* Wq, const float* sw, const uint16_t* bias, void* out,
                int64_t M, int64_t N, int64_t K, int64_t ldo, int out_s32, int path, cudaStream_t stream) {
   DeviceInfo* dev = nullptr;
   int st = current_device(&dev);
   if (st != W4A4_OK) return st;
   if (M == 0) return W4A4_OK;
+  if (path == 2) {
+    CUtensorMap tmA, tmB;
+    if ((st = packed_map(&tmA, Xq, M, K, 128, true)) != W4A4_OK) return st;
+    if ((st = packed_map(&tmB, Wq, N, K, 128, true)) != W4A4_OK) return st;
+    return gemm_legacy_launch(tmA, tmB, static_cast<int32_t*>(out), M, N, K, ldo, dev->status, stream) == cudaSuccess
+               ? W4A4_OK
+               : W4A4_ERR_CUDA;
+  }
   if (path == 1) {
     CUtensorMap tmW, tmX;
     if ((st = packed_map(&tmW, Wq, N, K, 128, true)) != W4A4_OK) return st;
@@ -318,7 +327,7 @@ int w4a4_gemm_s32(const int8_t* Xq, const int8_t* Wq, int32_t* acc, int64_t M, i
                   int path, void* workspace, size_t workspace_bytes, void* stream) {
   int st = validate_linear(Xq, nullptr, Wq, nullptr, nullptr, acc, M, N, K, ldc, 1);
   if (st != W4A4_OK) return st;
-  if (path != 0 && path != 1) return W4A4_ERR_ARG;
+  if (path != 0 && path != 1 && path != 2) return W4A4_ERR_ARG;
   if (path == 1 && M > kSmallMMax) return W4A4_ERR_SHAPE;
   (void)workspace;
   (void)workspace_bytes;

@@ -52,6 +52,11 @@ struct GemmArgs {
 // Launched as clusters of 2 CTAs.
 cudaError_t gemm_tc_launch(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmY, const GemmArgs& a,
                            int num_sms, cudaStream_t stream);
+// Comparison kernel in the pages' warp-level mma.m16n8k64.s4 design (raw int32
+// accumulators only); tmA / tmB: packed operands, box {64 bytes, 128 rows},
+// 64-byte swizzle.
+cudaError_t gemm_legacy_launch(const CUtensorMap& tmA, const CUtensorMap& tmB, int32_t* out, int64_t M, int64_t N,
+                               int64_t K, int64_t ldo, unsigned int* status, cudaStream_t stream);
 constexpr int kGemmBM = 256;
 constexpr int kGemmBN = 256;
 
