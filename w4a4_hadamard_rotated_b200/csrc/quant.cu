@@ -44,12 +44,24 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <cmath>
 #include <cstdint>
+#include <cstring>
+#include <mutex>
 
 #include "ptx.cuh"
 #include "w4a4_internal.h"
 
 namespace w4a4 {
+
+// GELU table: Phi(t), the standard normal CDF, for the bf16 values t with
+// exponent field kGeluFirstExp .. kGeluFirstExp + kGeluExps - 1
+// (2^-12 <= |t| < 8), 128 mantissas each, positive then negative.
+constexpr uint32_t kGeluFirstExp = 115;
+constexpr uint32_t kGeluExps = 15;
+constexpr int kGeluHalf = static_cast<int>(kGeluExps * 128);
+constexpr int kGeluTableSize = 2 * kGeluHalf;
+__device__ float g_gelu_table[kGeluTableSize];
 
 constexpr int kSlab = 64;      // elements per thread
 constexpr int kHalf = 32;      // packed pairs per thread
@@ -90,8 +102,29 @@ __device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
   return r;
 }
 
-__device__ __forceinline__ float gelu_erf(float t) {
-  return 0.5f * t * (1.0f + erff(t * 0.70710678118654752f));
+// GELU of the two bf16 inputs held in one 32-bit word: GELU(t) = t Phi(t)
+// with Phi(t) = (1 + erf(t / sqrt 2)) / 2 read from the table (one product,
+// so within about an ulp of the exact value).  The index is formed for both
+// halves at once with 16-bit SIMD min/max; clamping the exponent field to the
+// table's range is the only special case: below 2^-12 the entry of 2^-12
+// stands in (Phi differs by < 1e-4, the product by < 3e-8 absolute), at or
+// above 8 the entry of 8 - 2^-4 does (Phi rounds to 1, and t Phi(t) for
+// t <= -8 is below 6e-16 |t|).  `tab` is the table in shared memory.
+__device__ __forceinline__ void gelu_phi_word(uint32_t w, const float* __restrict__ tab, float& phi0, float& phi1) {
+  constexpr uint32_t lo = kGeluFirstExp << 7, hi = ((kGeluFirstExp + kGeluExps) << 7) - 1u;
+  uint32_t c;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(c) : "r"(w & 0x7FFF7FFFu), "r"(lo * 0x10001u));
+  asm("min.u16x2 %0, %0, %1;" : "+r"(c) : "r"(hi * 0x10001u));
+  // entry of each half: (c - lo) + sign * kGeluHalf; no half overflows 16 bits
+  const uint32_t idx = c - lo * 0x10001u + ((w >> 15) & 0x00010001u) * static_cast<uint32_t>(kGeluHalf);
+  phi0 = tab[idx & 0xFFFFu];
+  phi1 = tab[idx >> 16];
+}
+
+// bf16 bits of element e of a 16-byte chunk.
+__device__ __forceinline__ uint32_t bits16(const uint4 w, int e) {
+  const uint32_t word = e < 2 ? w.x : (e < 4 ? w.y : (e < 6 ? w.z : w.w));
+  return (e & 1) ? (word >> 16) : (word & 0xFFFFu);
 }
 
 // Element e of a 16-byte chunk as fp32.
@@ -117,6 +150,11 @@ __device__ __forceinline__ void fht_stage2(uint64_t (&V)[kHalf]) {
   }
 }
 
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
 __device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
   uint64_t r;
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
@@ -161,6 +199,7 @@ __global__ void __maxnreg__(96)
   constexpr int NCH = kSlab / C;   // 16-byte chunks per slab
 
   extern __shared__ __align__(128) uint8_t ring[];
+  __shared__ float gelu_tab[ACT == 1 ? kGeluTableSize : 1];
   __shared__ uint64_t full[kMaxStages];
   __shared__ unsigned int row_amax[3][kMaxRows];
   __shared__ int abort_flag;
@@ -183,6 +222,8 @@ __global__ void __maxnreg__(96)
   // waits for this grid's writes before it reads them
   griddep_launch_dependents();
   for (int i = tid; i < 3 * kMaxRows; i += blockDim.x) (&row_amax[0][0])[i] = 0u;
+  if (ACT == 1)
+    for (int i = tid; i < kGeluTableSize; i += blockDim.x) gelu_tab[i] = g_gelu_table[i];
   if (tid == 0) {
     for (int i = 0; i < kMaxStages; ++i) mbar_init(&full[i], 1);
     abort_flag = 0;
@@ -240,13 +281,16 @@ __global__ void __maxnreg__(96)
         }
 #pragma unroll
         for (int e = 0; e < C; ++e) {
-          float a = elem(lo, e, x);
-          float b = elem(hi, e, x);
-          if (ACT == 1) {
-            a = gelu_erf(a);
-            b = gelu_erf(b);
+          V[j * C + e] = pk2(elem(lo, e, x), elem(hi, e, x));
+          if (ACT == 1 && (e & 1)) {
+            // GELU = t * Phi(t): the Phi of elements e-1, e of both chunks
+            // come from one table lookup per 32-bit word
+            float pa0, pa1, pb0, pb1;
+            gelu_phi_word(bits16(lo, e - 1) | (bits16(lo, e) << 16), gelu_tab, pa0, pa1);
+            gelu_phi_word(bits16(hi, e - 1) | (bits16(hi, e) << 16), gelu_tab, pb0, pb1);
+            V[j * C + e - 1] = mul2(V[j * C + e - 1], pk2(pa0, pb0));
+            V[j * C + e] = mul2(V[j * C + e], pk2(pa1, pb1));
           }
-          V[j * C + e] = pk2(a, b);
         }
       }
     }
@@ -342,6 +386,36 @@ __global__ void __maxnreg__(96)
   }
 }
 
+// Fills the GELU table of the current device once: every bf16 t with
+// 2^-12 <= |t| < 8 gets fp32(Phi(t)) = fp32((1 + erf(t / sqrt 2)) / 2)
+// evaluated in double precision.  The copy is synchronous, so the first GELU call on a
+// device must not be inside a stream capture.
+static cudaError_t ensure_gelu_table() {
+  static bool ready[64] = {};
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (ready[dev]) return cudaSuccess;
+  static float host[kGeluTableSize];
+  for (int sgn = 0; sgn < 2; ++sgn)
+    for (uint32_t ex = 0; ex < kGeluExps; ++ex)
+      for (uint32_t f = 0; f < 128; ++f) {
+        const uint32_t bits = (static_cast<uint32_t>(sgn) << 15) | ((kGeluFirstExp + ex) << 7) | f;
+        const uint32_t fb = bits << 16;
+        float tf;
+        std::memcpy(&tf, &fb, sizeof(tf));
+        const double t = static_cast<double>(tf);
+        host[sgn * kGeluHalf + ex * 128 + f] = static_cast<float>(0.5 * (1.0 + std::erf(t / std::sqrt(2.0))));
+      }
+  e = cudaMemcpyToSymbol(g_gelu_table, host, sizeof(host));
+  if (e != cudaSuccess) return e;
+  ready[dev] = true;
+  return cudaSuccess;
+}
+
 // Registers per thread of one kernel instantiation (queried once).
 template <typename TIn, int G, int ACT>
 static int kernel_regs() {
@@ -366,7 +440,7 @@ struct RqPlan {
 // estimated time of the busiest SM: the rows it holds, divided by the warps
 // that share them (up to 16, beyond which an SM is saturated) and by the
 // fraction of lanes that carry a slab.
-static RqPlan plan_rq(int64_t M, int K, size_t elem_bytes, int regs, int num_sms) {
+static RqPlan plan_rq(int64_t M, int K, size_t elem_bytes, int regs, int num_sms, size_t static_bytes) {
   const int S = K / kSlab;
   const size_t row_bytes = static_cast<size_t>(K) * elem_bytes;
   const int regs_warp = (regs * 32 + 255) / 256 * 256;
@@ -381,7 +455,8 @@ static RqPlan plan_rq(int64_t M, int K, size_t elem_bytes, int regs, int num_sms
     if (cps > 8) cps = 8;
     const int64_t tiles = (M + P - 1) / P;
     for (int c = 1; c <= cps; ++c) {
-      int nst = static_cast<int>(kRingBytesPerSm / (static_cast<size_t>(c) * P * row_bytes));
+      const size_t ring_budget = kRingBytesPerSm > c * static_bytes ? kRingBytesPerSm - c * static_bytes : 0;
+      int nst = static_cast<int>(ring_budget / (static_cast<size_t>(c) * P * row_bytes));
       if (nst > kMaxStages) nst = kMaxStages;
       if (nst < kMinStages) break;
       const int64_t grid = tiles < static_cast<int64_t>(num_sms) * c ? tiles : static_cast<int64_t>(num_sms) * c;
@@ -408,7 +483,8 @@ static cudaError_t launch_rq(const TIn* x, int64_t M, int K, int64_t ldx, int8_t
                              unsigned int* status, cudaStream_t stream) {
   const int S = K / kSlab;
   if (S < 1 || S > kMaxThreads) return cudaErrorInvalidValue;
-  const RqPlan pl = plan_rq(M, K, sizeof(TIn), kernel_regs<TIn, G, ACT>(), num_sms);
+  const RqPlan pl = plan_rq(M, K, sizeof(TIn), kernel_regs<TIn, G, ACT>(), num_sms,
+                            ACT == 1 ? kGeluTableSize * sizeof(float) : 0);
   if (pl.P < 1) return cudaErrorInvalidValue;
   const size_t smem = static_cast<size_t>(pl.nst) * pl.P * K * sizeof(TIn);
   auto kern = rotate_quant_pack_kernel<TIn, G, ACT>;
@@ -436,6 +512,10 @@ static cudaError_t dispatch_rq(const TIn* x, int64_t M, int K, int64_t ldx, int 
 
 cudaError_t rotate_quant_bf16(const uint16_t* x, int64_t M, int K, int64_t ldx, int g, int act, int8_t* out,
                               float* scale, int num_sms, unsigned int* status, cudaStream_t stream) {
+  if (act == 1) {
+    const cudaError_t e = ensure_gelu_table();
+    if (e != cudaSuccess) return e;
+  }
   return dispatch_rq<uint16_t>(x, M, K, ldx, g, act, out, scale, num_sms, status, stream);
 }
 
