@@ -75,7 +75,10 @@ int w4a4_quantize_weight(const float* W, int64_t N, int64_t K, int64_t ldw, int 
  * quantize + pack in one pass" kernel of the page's Description).
  *   x   [M, K] bf16 bits, row stride ldx >= K, 16-byte aligned, ldx % 8 == 0
  *   act 0: none; 1: exact-erf GELU applied to x before the rotation (used to
- *       feed an MLP down projection from the up projection's output)
+ *       feed an MLP down projection from the up projection's output).  The
+ *       first act = 1 call on a device uploads a table of the normal CDF
+ *       (15 KB, synchronously); make that first call before any stream
+ *       capture.
  *   Xq  [M, K/2] int8 output (contiguous rows, 16-byte aligned); sx [M] fp32
  *   M >= 0 (M == 0 is a no-op); K % 128 == 0, K % g == 0, 128 <= K <= 32768.
  * A row that is all zero gets sx = 0 and all-zero codes.
