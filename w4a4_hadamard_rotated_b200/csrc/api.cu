@@ -145,7 +145,8 @@ int check_gemm_shape(int64_t M, int64_t N, int64_t K) {
 // tcgen05 tensor-core kernel; 1: the small-M weight-streaming kernel; 2: the
 // warp-level mma.sync comparison kernel (int32 output only).
 int run_linear(const int8_t* Xq, const float* sx, const int8_t* Wq, const float* sw, const uint16_t* bias, void* out,
-               int64_t M, int64_t N, int64_t K, int64_t ldo, int out_s32, int path, cudaStream_t stream) {
+               int64_t M, int64_t N, int64_t K, int64_t ldo, int out_s32, int path, cudaStream_t stream,
+               int early_w = 0) {
   DeviceInfo* dev = nullptr;
   int st = current_device(&dev);
   if (st != W4A4_OK) return st;
@@ -175,6 +176,7 @@ int run_linear(const int8_t* Xq, const float* sx, const int8_t* Wq, const float*
     a.ldo = ldo;
     a.out_s32 = out_s32;
     a.status = dev->status;
+    a.early_w = early_w;
     return smallm_launch_tm(tmW, tmX, a, stream) == cudaSuccess ? W4A4_OK : W4A4_ERR_CUDA;
   }
   CUtensorMap tmA, tmB, tmY;
@@ -361,7 +363,10 @@ int w4a4_linear_fused(const uint16_t* x, int64_t ldx, const int8_t* Wq, const fl
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if ((st = w4a4_quantize_activation(x, M, K, ldx, g, act, xq, sx, stream)) != W4A4_OK) return st;
   const int path = (M <= smallm_threshold()) ? 1 : 0;
-  return run_linear(xq, sx, Wq, sw, bias, y, M, N, K, ldy, 0, path, s);
+  // The quantiser above is launched in plain stream order, so whatever wrote
+  // the weights finished before it started: the small-M kernel may begin
+  // streaming them before its grid-dependency wait.
+  return run_linear(xq, sx, Wq, sw, bias, y, M, N, K, ldy, 0, path, s, 1);
 }
 
 int w4a4_last_device_error(void* stream) {

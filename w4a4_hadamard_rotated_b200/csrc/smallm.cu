@@ -24,11 +24,12 @@
 //     (1,3,5,7, 0,2,4,6) for both operands, so the MMA accumulates 256*acc.
 //   * The K slices of one weight tile run as one cluster of up to 8 CTAs.
 //     Each CTA parks its int32 partial tile in its shared memory; after a
-//     cluster barrier, CTA c reads its share of the tile's rows from every
-//     CTA of the cluster (distributed shared memory), sums them in rank order
-//     (integer addition: exact and deterministic), applies the epilogue and
-//     writes y.  The reduction never leaves the chip, and the kernel needs no
-//     workspace.
+//     cluster barrier it pushes the rows every other CTA owns into that
+//     CTA's shared memory with one bulk copy per owner (distributed shared
+//     memory, completing on the owner's barrier).  CTA c sums its share of
+//     the rows (integer addition: exact in any order), applies the epilogue
+//     and writes y.  The reduction never leaves the chip, and the kernel
+//     needs no workspace.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -50,6 +51,7 @@ constexpr int kGroups = 2;     // widen groups of kWorkWarps warps, taking turns
 constexpr int kThreads = (2 + kGroups * kWorkWarps) * 32;
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kTmemA = 64;   // first widened-weight column (the accumulator takes NP <= 64)
+constexpr int kMaxSplits = 8;     // K slices per weight tile at most (the portable cluster size)
 
 // Two CTAs share an SM, so each keeps its rings within ~110 KB of shared
 // memory: NP = 64 (8 KB widened activations per stage) takes shallower rings.
@@ -66,6 +68,13 @@ struct Layout {
   static constexpr uint32_t kBytes = kOffPackX + kSP * kPackX;
   static constexpr uint32_t kAlloc = kBytes + 1024;
   static_assert(kOffPackW % 1024 == 0, "alignment");
+  // After the main loop: the parked partial tile (WM rows x NP int32) and the
+  // receive slots of the split-K reduction (at most WM + kMaxSplits rows), both
+  // in the idle ring memory.
+  static constexpr int kChunkMask = (NP / 4 < 8 ? NP / 4 : 8) - 1;
+  static constexpr uint32_t kOffPark = 0;
+  static constexpr uint32_t kOffRecv = kOffPark + WM * NP * 4;
+  static_assert(kOffRecv + (WM + kMaxSplits) * NP * 4 <= kBytes, "reduction buffers fit in the rings");
 };
 
 struct Bars {
@@ -77,6 +86,7 @@ struct Bars {
   uint64_t wfull[ST];    // kWorkWarps arrivals (widened stage written)
   uint64_t wempty[ST];   // one MMA commit
   uint64_t acc_full;
+  uint64_t recv_full;    // the other K slices' rows of this CTA's share (split-K reduction)
   uint32_t tmem_base;
   int abort_flag;
   unsigned int last;
@@ -137,18 +147,18 @@ __device__ __forceinline__ void tmem_ld_cols<64>(uint32_t taddr, uint32_t (&r)[6
   tmem_ld_32x32b_x32(taddr + 32, b);
 }
 
-// 32-bit load from the shared memory of CTA `rank` of this cluster, at the
-// offset that `local` (a shared::cta address) has in this CTA.
-__device__ __forceinline__ int32_t ld_shared_cluster_s32(uint32_t local, uint32_t rank) {
-  int32_t v;
+// Bulk copy of `bytes` (a multiple of 16; both addresses 16-byte aligned)
+// from this CTA's shared memory at `src` to CTA `rank` of this cluster at the
+// shared::cta offset `dst`; the transfer completes on the barrier at offset
+// `bar` in CTA `rank`.
+__device__ __forceinline__ void bulk_push(uint32_t dst, uint32_t src, uint32_t bytes, uint32_t bar, uint32_t rank) {
   asm volatile(
-      "{\n\t.reg .b32 ra;\n\t"
-      "mapa.shared::cluster.u32 ra, %1, %2;\n\t"
-      "ld.shared::cluster.s32 %0, [ra];\n\t}"
-      : "=r"(v)
-      : "r"(local), "r"(rank)
+      "{\n\t.reg .b32 rd, rb;\n\t"
+      "mapa.shared::cluster.u32 rd, %0, %4;\n\t"
+      "mapa.shared::cluster.u32 rb, %3, %4;\n\t"
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [rd], [%1], %2, [rb];\n\t}" ::"r"(dst),
+      "r"(src), "r"(bytes), "r"(bar), "r"(rank)
       : "memory");
-  return v;
 }
 
 __device__ __forceinline__ float bf16_to_f(uint16_t b) { return __uint_as_float(static_cast<uint32_t>(b) << 16); }
@@ -186,30 +196,36 @@ __global__ void __launch_bounds__(kThreads, 2)
       mbar_init(&bars.wempty[s], 1);
     }
     mbar_init(&bars.acc_full, 1);
+    mbar_init(&bars.recv_full, 1);
     bars.abort_flag = 0;
     fence_mbar_init();
+    fence_async_shared();   // the barriers are visible to the copy engine
     tma_prefetch_desc(&tmW);
     tma_prefetch_desc(&tmX);
+    if (args.early_w) {
+      // The packed weights were written before the previous kernel of the
+      // stream started (the caller guarantees it), so their first ring
+      // stages stream in from the first cycle, before tensor memory is
+      // allocated and before the previous kernel has finished.
+      const int pre = min(Lay::kSP, nkb);
+      for (int i = 0; i < pre; ++i) {
+        mbar_arrive_expect_tx(&bars.full[i], Lay::kPackW + Lay::kPackX);
+        tma_load_2d(smem + Lay::kOffPackW + i * Lay::kPackW, &tmW, &bars.full[i], (kb0 + i) * BKP, ntile * WM);
+      }
+    }
   }
   if (warp == 1) {
     tmem_alloc(&bars.tmem_base, kTmemCols);
     tmem_relinquish();
   }
+  // A kernel launched after this one with programmatic stream serialization
+  // may start its own set-up now; it reads nothing this kernel writes before
+  // its grid-dependency wait, which returns only once this grid has finished.
+  griddep_launch_dependents();
   // launched with programmatic stream serialization: the set-up above may
   // overlap the previous kernel (the activation quantiser of a fused layer);
   // its outputs are read only after this point
   griddep_wait();
-  if (!OUT_S32 && warp >= 2) {
-    // epilogue operands, loaded now so that their latency hides behind the stream
-    const int t = threadIdx.x - 64;
-    if (t < WM) {
-      const int64_t n = static_cast<int64_t>(ntile) * WM + t;
-      bars.sw[t] = n < N ? args.sw[n] : 0.0f;
-      bars.bias[t] = (n < N && args.bias != nullptr) ? bf16_to_f(args.bias[n]) : 0.0f;
-    } else if (t < WM + 64) {
-      bars.sx[t - WM] = t - WM < M ? args.sx[t - WM] : 0.0f;
-    }
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -222,10 +238,13 @@ __global__ void __launch_bounds__(kThreads, 2)
       uint32_t ps = 0, ph = 0;
       int issued = 0;
       bool ok = true;
+      const int pre = args.early_w ? min(Lay::kSP, nkb) : 0;   // weight stages already in flight
       for (int kb = kb0; kb < kb1; ++kb) {
-        if (!mbar_wait(&bars.empty[ps], ph ^ 1, abort_flag, args.status)) { ok = false; break; }
-        mbar_arrive_expect_tx(&bars.full[ps], Lay::kPackW + Lay::kPackX);
-        tma_load_2d(smem + Lay::kOffPackW + ps * Lay::kPackW, &tmW, &bars.full[ps], kb * BKP, ntile * WM);
+        if (kb - kb0 >= pre) {
+          if (!mbar_wait(&bars.empty[ps], ph ^ 1, abort_flag, args.status)) { ok = false; break; }
+          mbar_arrive_expect_tx(&bars.full[ps], Lay::kPackW + Lay::kPackX);
+          tma_load_2d(smem + Lay::kOffPackW + ps * Lay::kPackW, &tmW, &bars.full[ps], kb * BKP, ntile * WM);
+        }
         tma_load_2d(smem + Lay::kOffPackX + ps * Lay::kPackX, &tmX, &bars.full[ps], kb * BKP, 0);
         ++issued;
         if (++ps == Lay::kSP) { ps = 0; ph ^= 1; }
@@ -263,6 +282,18 @@ __global__ void __launch_bounds__(kThreads, 2)
     // unit u (16 packed bytes) is part u % 4 of row u / 4; its 32 widened
     // bytes go to chunks 2 * part and 2 * part + 1 of that row in the
     // 128-byte-swizzle K-major layout of the B operand.
+    if (!OUT_S32) {
+      // epilogue operands; read only after the cluster barrier that precedes
+      // the reduction, so their latency hides behind the weight stream
+      const int t = threadIdx.x - 64;
+      if (t < WM) {
+        const int64_t n = static_cast<int64_t>(ntile) * WM + t;
+        bars.sw[t] = n < N ? args.sw[n] : 0.0f;
+        bars.bias[t] = (n < N && args.bias != nullptr) ? bf16_to_f(args.bias[n]) : 0.0f;
+      } else if (t < WM + 64) {
+        bars.sx[t - WM] = t - WM < M ? args.sx[t - WM] : 0.0f;
+      }
+    }
     const int q = warp & 3;
     const int r = q * 32 + lane;
     const int grp = (warp - 2) / kWorkWarps;
@@ -316,9 +347,10 @@ __global__ void __launch_bounds__(kThreads, 2)
         mbar_arrive(&bars.empty[ps]);
       }
     }
-    // The first group moves this CTA's partial tile from tensor memory to
-    // shared memory (the packed-weight ring, idle once the accumulator is
-    // complete), laid out part[m][r] so that a warp's rows are contiguous.
+    // The first group parks this CTA's partial tile in shared memory (the
+    // rings are idle once the accumulator is complete): row r of the tile is
+    // NP consecutive int32 values, its 16-byte chunk j stored at chunk
+    // j ^ (r & kChunkMask), so the rows that go to one owner are contiguous.
     if (grp == 0) {
       if (ok) (void)warp_wait(&bars.acc_full, 0, abort_flag, args.status);
       if (*abort_flag == 0) {
@@ -326,45 +358,84 @@ __global__ void __launch_bounds__(kThreads, 2)
         uint32_t acc[NP];
         tmem_ld_cols<NP>(tmem_base + (static_cast<uint32_t>(q * 32) << 16), acc);
         tmem_wait_ld();
-        int32_t* part = reinterpret_cast<int32_t*>(smem + Lay::kOffPackW);
+        uint8_t* row = smem + Lay::kOffPark + r * (NP * 4);
 #pragma unroll
-        for (int m = 0; m < NP; ++m) part[m * WM + r] = static_cast<int32_t>(acc[m]) >> 8;
+        for (int j = 0; j < NP / 4; ++j) {
+          const int4 c = make_int4(static_cast<int32_t>(acc[4 * j]) >> 8, static_cast<int32_t>(acc[4 * j + 1]) >> 8,
+                                   static_cast<int32_t>(acc[4 * j + 2]) >> 8, static_cast<int32_t>(acc[4 * j + 3]) >> 8);
+          *reinterpret_cast<int4*>(row + ((j ^ (r & Lay::kChunkMask)) << 4)) = c;
+        }
+        fence_async_shared();   // read next by bulk copies
       }
     }
   }
 
   // ---- K-slice reduction across the cluster (one cluster per weight tile,
-  // one CTA per K slice), through distributed shared memory: CTA c sums rows
-  // [c*R, c*R + R) of the tile over the cluster's partials in rank order
-  // (integer addition: exact and deterministic), applies the epilogue and
-  // writes those outputs.
+  // one CTA per K slice).  CTA c owns rows [c*R, c*R + R) of the tile.  After
+  // a cluster barrier (every CTA's rings are idle and its partial tile is
+  // parked) each CTA pushes the rows every other CTA owns into that CTA's
+  // receive slot for this rank with one bulk copy, which completes on the
+  // owner's barrier; the owner sums its own rows and the received ones
+  // (integer addition: exact in any order), applies the epilogue and writes
+  // those outputs.  Nothing is read remotely, so no second barrier is needed:
+  // an owner leaves only once every byte sent to it has landed, and a sender
+  // only once its copies have read its shared memory.
+  const int R = (WM + splits - 1) / splits;
+  const int own_rows = min(WM - split * R, R);
+  const uint32_t slot_bytes = static_cast<uint32_t>(R) * NP * 4;
+  if (threadIdx.x == 0 && splits > 1)
+    mbar_arrive_expect_tx(&bars.recv_full, static_cast<uint32_t>(splits - 1) * own_rows * NP * 4);
   tc_fence_before();
   __syncthreads();
-  cluster_sync();   // every CTA's partial tile is in its shared memory
-  {
-    const int R = (WM + splits - 1) / splits;
-    const int r0 = split * R;
-    const int rows = min(WM - r0, R);
-    const int mrows = static_cast<int>(M);
-    const uint32_t part_local = smem_u32(smem + Lay::kOffPackW);
-    for (int idx = threadIdx.x; idx < rows * mrows; idx += kThreads) {
-      const int m = idx / rows;
-      const int rr = r0 + (idx - m * rows);
+  cluster_sync();   // every CTA of the cluster is done with its rings and has parked its partial tile
+  if (threadIdx.x == 0 && splits > 1) {
+    for (int c = 0; c < splits; ++c) {
+      if (c == split) continue;
+      const int rows_c = min(WM - c * R, R);
+      bulk_push(smem_u32(smem + Lay::kOffRecv) + split * slot_bytes,
+                smem_u32(smem + Lay::kOffPark) + static_cast<uint32_t>(c) * slot_bytes,
+                static_cast<uint32_t>(rows_c) * NP * 4, smem_u32(&bars.recv_full), static_cast<uint32_t>(c));
+    }
+    bulk_commit_group();
+  }
+  bool got = true;
+  if (splits > 1) got = warp_wait(&bars.recv_full, 0, abort_flag, args.status);
+  if (got && *abort_flag == 0) {
+    // item = (owned row, chunk of four activation rows); consecutive threads
+    // take consecutive rows, so the stores of one activation row coalesce
+    const int chunks = (static_cast<int>(M) + 3) / 4;
+    for (int it = threadIdx.x; it < own_rows * chunks; it += kThreads) {
+      const int j = it / own_rows;
+      const int rl = it - j * own_rows;
+      const int rr = split * R + rl;   // row in the tile
+      const uint32_t coff = static_cast<uint32_t>(((j ^ (rr & Lay::kChunkMask)) << 4));
+      int4 sum = *reinterpret_cast<const int4*>(smem + Lay::kOffPark + rr * (NP * 4) + coff);
+      for (int c = 0; c < splits; ++c) {
+        if (c == split) continue;
+        const int4 v = *reinterpret_cast<const int4*>(smem + Lay::kOffRecv + c * slot_bytes + rl * (NP * 4) + coff);
+        sum.x += v.x;
+        sum.y += v.y;
+        sum.z += v.z;
+        sum.w += v.w;
+      }
       const int64_t n = static_cast<int64_t>(ntile) * WM + rr;   // weight row = output column
       if (n >= N) continue;
-      const uint32_t off = static_cast<uint32_t>(m * WM + rr) * 4u;
-      int32_t sum = 0;
-      for (int c = 0; c < splits; ++c) sum += ld_shared_cluster_s32(part_local + off, static_cast<uint32_t>(c));
-      if (OUT_S32) {
-        reinterpret_cast<int32_t*>(args.out)[static_cast<int64_t>(m) * args.ldo + n] = sum;
-      } else {
-        float y = __fmul_rn(__fmul_rn(__int2float_rn(sum), bars.sx[m]), bars.sw[rr]);
-        if (args.bias != nullptr) y = __fadd_rn(y, bars.bias[rr]);
-        reinterpret_cast<uint16_t*>(args.out)[static_cast<int64_t>(m) * args.ldo + n] = f_to_bf16(y);
+      const int32_t s4[4] = {sum.x, sum.y, sum.z, sum.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int64_t m = 4 * j + e;
+        if (m >= M) break;
+        if (OUT_S32) {
+          reinterpret_cast<int32_t*>(args.out)[m * args.ldo + n] = s4[e];
+        } else {
+          float y = __fmul_rn(__fmul_rn(__int2float_rn(s4[e]), bars.sx[m]), bars.sw[rr]);
+          if (args.bias != nullptr) y = __fadd_rn(y, bars.bias[rr]);
+          reinterpret_cast<uint16_t*>(args.out)[m * args.ldo + n] = f_to_bf16(y);
+        }
       }
     }
   }
-  cluster_sync();   // no CTA leaves while its partial tile may still be read
+  if (threadIdx.x == 0 && splits > 1) bulk_wait_group_read<0>();   // the pushes have read the parked tile
   if (warp == 1) {
     // the MMA thread's final commit arrives when every MMA has completed
     if (lane == 0) (void)mbar_wait(&bars.acc_full, 0, nullptr, nullptr, 100000000ull);
@@ -373,8 +444,6 @@ __global__ void __launch_bounds__(kThreads, 2)
     tmem_dealloc(tmem_base, kTmemCols);
   }
 }
-
-constexpr int kMaxSplits = 8;   // the portable cluster size
 
 template <int NP, int OUT_S32>
 void fill_cfg(cudaLaunchConfig_t* cfg, cudaLaunchAttribute* attr, int ctas, int splits, cudaStream_t stream) {
