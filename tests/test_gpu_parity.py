@@ -30,6 +30,11 @@ def _packed_cuda(q):
 @pytest.mark.parametrize("M,K,g,act", [
     (16, 256, 128, 0), (333, 3072, 128, 0), (333, 3072, 64, 0), (333, 3072, 256, 0),
     (67, 12288, 128, 0), (67, 12288, 256, 1), (130, 5120, 64, 1), (1, 128, 128, 0), (5, 13824, 128, 0),
+    # 512 rows and more without activation take the tensor-core rotation (the
+    # threshold the test session sets)
+    # (whole rows per 128-lane tile: 5 x 24, 1 x 96, 3 x 40, 1 x 108, 2 x 48 lanes)
+    (777, 3072, 128, 0), (520, 12288, 128, 0), (513, 5120, 128, 0), (1000, 13824, 128, 0), (600, 3072, 64, 0),
+    (700, 256, 128, 0),
 ])
 def test_quantize_activation_parity(cuda_lib, M, K, g, act):
     x = workloads.make_activation(M, K, seed=M + K + g, outlier_frac=0.005, outlier_scale=30.0)
@@ -38,8 +43,9 @@ def test_quantize_activation_parity(cuda_lib, M, K, g, act):
     check_packed(Xq, sx, ref, f"x {M}x{K} g{g} act{act}")
 
 
-def test_quantize_activation_strided_rows(cuda_lib):
-    M, K, g = 70, 1024, 128
+@pytest.mark.parametrize("M", [70, 700])
+def test_quantize_activation_strided_rows(cuda_lib, M):
+    K, g = 1024, 128
     wide = workloads.make_activation(M, K + 64, seed=3, outlier_frac=0.01, outlier_scale=20.0).cuda()
     x = wide[:, :K]
     Xq, sx = cuda_lib.quantize_activation(x, g)
@@ -274,7 +280,8 @@ def test_bounded_wait_reports_timeout_and_context_survives(cuda_lib):
     _check_layer(cuda_lib, cfg, x, W, b)
 
 
-def test_quantize_exact_ties_follow_round_half_even(cuda_lib):
+@pytest.mark.parametrize("n_rows", [300, 600])
+def test_quantize_exact_ties_follow_round_half_even(cuda_lib, n_rows):
     """Rows built from the hand-derived tie fixture: every rotated value is an
     exact multiple of 1/2 or 1/4, so many codes sit exactly on a rounding
     boundary.  The kernel must decide all of them as round-half-even of the
@@ -292,7 +299,7 @@ def test_quantize_exact_ties_follow_round_half_even(cuda_lib):
     # K = 128 (two groups of 64): pair the cases, and repeat with permuted
     # group order and signs so the rows span several CTAs and lanes
     base = [np.concatenate([rows[0], rows[1]]), np.concatenate([rows[1], -rows[0]])]
-    X = np.stack([base[i % 2] * (1 if (i // 2) % 2 == 0 else -1) for i in range(300)])
+    X = np.stack([base[i % 2] * (1 if (i // 2) % 2 == 0 else -1) for i in range(n_rows)])
     xb = orc.f32_to_bf16_bits(X.astype(np.float32))
     assert np.array_equal(orc.bf16_bits_to_f32(xb).astype(np.float64), X)
     x = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).cuda()

@@ -91,6 +91,23 @@ int packed_map(CUtensorMap* map, const int8_t* base, int64_t rows, int64_t K, in
   return r == CUDA_SUCCESS ? W4A4_OK : W4A4_ERR_CUDA;
 }
 
+// 3-D map over bf16 rows x [M, K] (row stride ldx elements) viewed as
+// [M][K/g][g]: box {64 elements, K/g groups, rows_per_tile rows}, 128-byte
+// swizzle, so one box lands as rows_per_tile * K/g consecutive 128-byte
+// rows (group j of row p at row p * K/g + j); rows past M read as zero.
+int group_rows_map(CUtensorMap* map, const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int g, int rows_per_tile) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return W4A4_ERR_CUDA;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(g), static_cast<cuuint64_t>(K / g), static_cast<cuuint64_t>(M)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(g) * 2, static_cast<cuuint64_t>(ldx) * 2};
+  const cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(K / g), static_cast<cuuint32_t>(rows_per_tile)};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t*>(x), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? W4A4_OK : W4A4_ERR_CUDA;
+}
+
 namespace {
 
 // 2-D map over a bf16 output [rows, cols] with row stride ld (elements), box

@@ -44,7 +44,9 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <climits>
 #include <cmath>
+#include <cstdlib>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -510,8 +512,38 @@ static cudaError_t dispatch_rq(const TIn* x, int64_t M, int K, int64_t ldx, int 
   return cudaErrorInvalidValue;
 }
 
+// The tensor-core rotation (quant_tc.cu) takes bf16 rows without activation
+// for g in {64, 128} and K / g <= 128, from rotate_tc_min_rows() rows up.
+// Measured on B200 (CUDA-graph replay): alone it is faster from a few
+// hundred rows up (4608 x 3072: 9.7 vs 11.1 us; 32760 x 5120: 64 vs 91 us),
+// but inside the fused layer, ahead of the GEMM, only the 32760-row shapes
+// gain (0.7%) while 4608-row layers lose 1-2 us, so by default it serves
+// batches of 8192 rows and more.  W4A4_ROTATE_TC_MIN_ROWS=<n> moves the
+// threshold (the test suite sets 512 so that its parity cases reach both
+// kernels); W4A4_ROTATE_TC=0 selects the register-butterfly kernel always.
+static int64_t rotate_tc_min_rows() {
+  static int64_t v = -1;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    v = 8192;
+    const char* off = std::getenv("W4A4_ROTATE_TC");
+    if (off != nullptr && off[0] == '0' && off[1] == '\0') {
+      v = INT64_MAX;
+      return;
+    }
+    const char* e = std::getenv("W4A4_ROTATE_TC_MIN_ROWS");
+    if (e != nullptr) {
+      const long long x = std::strtoll(e, nullptr, 10);
+      if (x >= 1) v = x;
+    }
+  });
+  return v;
+}
+
 cudaError_t rotate_quant_bf16(const uint16_t* x, int64_t M, int K, int64_t ldx, int g, int act, int8_t* out,
                               float* scale, int num_sms, unsigned int* status, cudaStream_t stream) {
+  if (act == 0 && (g == 64 || g == 128) && K / g <= 128 && M >= rotate_tc_min_rows())
+    return rotate_quant_bf16_tc(x, M, K, ldx, g, out, scale, num_sms, status, stream);
   if (act == 1) {
     const cudaError_t e = ensure_gelu_table();
     if (e != cudaSuccess) return e;

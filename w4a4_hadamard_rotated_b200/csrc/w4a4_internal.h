@@ -20,6 +20,9 @@ int current_device(DeviceInfo** out);
 // TMA map over a packed int4 matrix [rows, K/2] bytes with box {64, box_rows}
 // (64-byte swizzle in shared memory when swizzle64).
 int packed_map(CUtensorMap* map, const int8_t* base, int64_t rows, int64_t K, int box_rows, bool swizzle64 = false);
+// TMA map over bf16 rows [M, K] (row stride ldx) viewed as [M][K/g][g], box
+// {64, K/g, rows_per_tile}, 128-byte swizzle (the tensor-core rotation's A tiles).
+int group_rows_map(CUtensorMap* map, const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int g, int rows_per_tile);
 // Argument checks of w4a4_linear (out_s32 = 0) / w4a4_gemm_s32 (out_s32 = 1).
 int validate_linear(const int8_t* Xq, const float* sx, const int8_t* Wq, const float* sw, const uint16_t* bias,
                     const void* y, int64_t M, int64_t N, int64_t K, int64_t ldy, int out_s32);
@@ -29,6 +32,10 @@ cudaError_t rotate_quant_bf16(const uint16_t* x, int64_t M, int K, int64_t ldx, 
                               float* scale, int num_sms, unsigned int* status, cudaStream_t stream);
 cudaError_t rotate_quant_f32(const float* x, int64_t M, int K, int64_t ldx, int g, int8_t* out, float* scale,
                              int num_sms, unsigned int* status, cudaStream_t stream);
+// Tensor-core form of rotate_quant_bf16 for act = 0, g in {64, 128} and
+// K / g <= 128 (quant_tc.cu); returns cudaErrorNotSupported for other shapes.
+cudaError_t rotate_quant_bf16_tc(const uint16_t* x, int64_t M, int K, int64_t ldx, int g, int8_t* out, float* scale,
+                                 int num_sms, unsigned int* status, cudaStream_t stream);
 // Largest K the in-register rotate kernel supports: 512 threads x 64 codes
 // per row for bf16 rows; fp32 rows (weights) are limited by two ring stages
 // of one row in shared memory (2 x 96 KB).
