@@ -27,6 +27,16 @@
  *   - Only sm_100 devices are supported (W4A4_ERR_DEVICE otherwise).
  *   - Calls are thread-safe as long as different host threads use different
  *     outputs and workspaces.
+ *
+ * Environment (read once per process, at the first call that needs it; they
+ * choose between kernels that compute the same result):
+ *   - W4A4_SMALLM_MAX=<0..64>: w4a4_linear_fused uses the small-M
+ *     weight-streaming kernel for M up to this value (default 64).
+ *   - W4A4_ROTATE_TC_MIN_ROWS=<n>: activations without GELU, g in {64, 128}
+ *     and K/g <= 128 are rotated on the tensor cores from n rows up (default
+ *     8192); W4A4_ROTATE_TC=0 keeps the register-butterfly kernel for every
+ *     shape.  The two differ only in the order of the fp32 additions of the
+ *     rotation.
  */
 #ifndef W4A4_H_
 #define W4A4_H_
