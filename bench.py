@@ -333,7 +333,9 @@ def run_impl(args, cfg, world, rank, local):
 
     # ---- per-kernel launch durations (the kernels and launch shapes the fused
     # call runs, on the launching stream) for the roofline of the dominant kernel
-    small = cfg.M <= 64
+    path = w4.linear_kernel(cfg.M, cfg.N, cfg.K)   # the GEMM kernel linear() runs here
+    small = path != 0
+    gemm_name = {0: "gemm_tc", 1: "smallm", 3: "gemv"}[path]
 
     def quant(i):
         s = sets[i % len(sets)]
@@ -419,8 +421,10 @@ def run_impl(args, cfg, world, rank, local):
         # weight streaming: the packed weight dominates the bytes
         k3_bytes = cfg.N * cfg.K // 2 + cfg.M * cfg.K // 2 + 4 * (cfg.M + cfg.N) + 2 * cfg.M * cfg.N
         roof = {"bound": "hbm", "achieved": k3_bytes / t_gemm / 1e9, "peak": hbm, "unit": "GB/s",
-                "frac": k3_bytes / t_gemm / 1e9 / hbm, "traffic": MEASURED_TRAFFIC.get(("smallm", args.workload)),
-                "kernel": "smallm_kernel (split-K weight streaming)", "peak_note": f"{kind} HBM copy"}
+                "frac": k3_bytes / t_gemm / 1e9 / hbm, "traffic": MEASURED_TRAFFIC.get((gemm_name, args.workload)),
+                "kernel": ("smallm_kernel (split-K weight streaming on the tensor cores)" if path == 1 else
+                           "gemv_kernel (weight streaming on the CUDA cores)"),
+                "peak_note": f"{kind} HBM copy"}
     else:
         roof = {"bound": "tensor", "achieved": gemm_tops, "peak": int8_peak, "unit": "TOPS",
                 "frac": gemm_tops / int8_peak, "traffic": MEASURED_TRAFFIC.get(("gemm_tc", args.workload)),
@@ -446,7 +450,7 @@ def run_impl(args, cfg, world, rank, local):
         "us_per_layer_eager_launches": dt_eager / args.steps * 1e6,
         "roofline_fraction_of_layer": roof_time / (ms_per_step / 1e3),
         "layer_roofline_us": roof_time * 1e6,
-        "kernels_us": {"rotate_quant_pack": t_quant * 1e6, ("smallm" if small else "gemm_tc"): t_gemm * 1e6},
+        "kernels_us": {"rotate_quant_pack": t_quant * 1e6, gemm_name: t_gemm * 1e6},
         "roofline": roof,
         "quant_kernel_roofline": {"bound": "hbm", "achieved": quant_bytes / t_quant / 1e9, "peak": hbm,
                                   "unit": "GB/s", "frac": quant_bytes / t_quant / 1e9 / hbm},

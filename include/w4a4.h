@@ -30,8 +30,9 @@
  *
  * Environment (read once per process, at the first call that needs it; they
  * choose between kernels that compute the same result):
- *   - W4A4_SMALLM_MAX=<0..64>: w4a4_linear_fused uses the small-M
- *     weight-streaming kernel for M up to this value (default 64).
+ *   - W4A4_SMALLM_MAX=<0..64>: w4a4_linear and w4a4_linear_fused use the
+ *     weight-streaming kernels for M up to this value (default 64); the
+ *     CUDA-core one serves M = 1 and M <= 4 with M*K <= 12288 of those.
  *   - W4A4_ROTATE_TC_MIN_ROWS=<n>: activations without GELU, g in {64, 128}
  *     and K/g <= 128 are rotated on the tensor cores from n rows up (default
  *     8192); W4A4_ROTATE_TC=0 keeps the register-butterfly kernel for every
@@ -107,9 +108,11 @@ int w4a4_quantize_activation(const uint16_t* x, int64_t M, int64_t K, int64_t ld
  *   M >= 0, N >= 1, N % 8 == 0, 32 <= K <= 131072, K % 32 == 0; Xq/Wq 16-byte aligned
  *   workspace, workspace_bytes: reserved; no kernel needs scratch memory
  *       (w4a4_workspace_bytes returns 0), so both may be NULL / 0.
- * M <= 64 takes the weight-streaming split-K kernel (K slices reduced on chip
- * within a CTA cluster), larger M the tcgen05 tensor-core kernel; both give
- * bit-identical int32 accumulators.
+ * M = 1, or M <= 4 with M*K <= 12288, takes a weight-streaming kernel on
+ * the CUDA cores (dp4a on widened nibbles), M <= 64 the weight-streaming split-K
+ * tensor-core kernel (K slices reduced on chip within a CTA cluster), larger
+ * M the tcgen05 tensor-core kernel; all give bit-identical int32
+ * accumulators.
  */
 int w4a4_linear(const int8_t* Xq, const float* sx, const int8_t* Wq, const float* sw,
                 const uint16_t* bias, uint16_t* y, int64_t M, int64_t N, int64_t K,
@@ -129,6 +132,13 @@ int w4a4_linear_fused(const uint16_t* x, int64_t ldx, const int8_t* Wq, const fl
                       int64_t K, int g, int act, void* workspace, size_t workspace_bytes,
                       void* stream);
 
+/* Which GEMM kernel w4a4_linear and w4a4_linear_fused run for this shape,
+ * numbered as w4a4_gemm_s32's path: 0 = tcgen05 tensor-core kernel, 1 =
+ * small-M split-K kernel, 3 = tiny-M CUDA-core kernel.  (w4a4_linear_noalloc,
+ * for M <= 64, runs 3 where this returns 3 and 1 otherwise.)  Pure host
+ * function; it reads the environment switches above. */
+int w4a4_linear_kernel(int64_t M, int64_t N, int64_t K);
+
 /* Workspace sizes in bytes (0 when none is needed: w4a4_workspace_bytes is
  * always 0).  Pure host functions. */
 size_t w4a4_workspace_bytes(int64_t M, int64_t N, int64_t K);
@@ -139,7 +149,9 @@ size_t w4a4_fused_workspace_bytes(int64_t M, int64_t N, int64_t K);
  * for bit-exact checks of the GEMM.  path: 0 = tcgen05 tensor-core kernel,
  * 1 = small-M weight-streaming kernel (M <= 64 only), 2 = a comparison
  * kernel in the pages' own design (warp-level mma.m16n8k64.s4 fed from
- * shared memory), kept to measure the tcgen05 kernel against.
+ * shared memory), kept to measure the tcgen05 kernel against, 3 = tiny-M
+ * CUDA-core weight-streaming kernel (M <= 4, M*K <= 96 KiB; W4A4_ERR_SHAPE
+ * otherwise).
  *   acc [M, N] int32 output with row stride ldc >= N, ldc % 4 == 0.
  * Other rules as for w4a4_linear.
  */
@@ -157,8 +169,10 @@ int w4a4_gemm_s32(const int8_t* Xq, const int8_t* Wq, int32_t* acc, int64_t M, i
  * synchronise the device and fragment a pool sized in advance).
  *   Arguments, layouts and results are those of w4a4_linear; the output is
  *   bit-identical to it.  The small-M kernel reduces its K slices in the
- *   shared memory of a CTA cluster, so no scratch memory of any kind is
- *   used: neither a caller workspace nor memory of the library's own.
+ *   shared memory of a CTA cluster, and the tiny-M kernel (M <= 4) keeps its
+ *   operands in one CTA's registers and shared memory, so no scratch memory
+ *   of any kind is used: neither a caller workspace nor memory of the
+ *   library's own.
  *   M > 64 gives W4A4_ERR_SHAPE before anything is launched.  Calls are
  *   independent (they may overlap on the GPU).
  */

@@ -98,9 +98,27 @@ def test_fused_rejects_bad_arguments(lib):
 
 def test_gemm_s32_rejects_bad_arguments(lib):
     f = lib.w4a4_gemm_s32
-    assert f(FAKE, FAKE, FAKE, 128, 256, 256, 256, 3, NULL, 0, NULL) == 9      # path
+    assert f(FAKE, FAKE, FAKE, 128, 256, 256, 256, 4, NULL, 0, NULL) == 9      # path
+    assert f(FAKE, FAKE, FAKE, 5, 256, 256, 256, 3, NULL, 0, NULL) == 2        # tiny-M path, M > 4
+    assert f(FAKE, FAKE, FAKE, 4, 256, 32768, 256, 3, NULL, 0, NULL) == 2      # tiny-M path, M*K > 96 KB
     assert f(FAKE, FAKE, FAKE, 65, 256, 256, 256, 1, NULL, 0, NULL) == 2       # small-M path, M > 64
     assert f(FAKE, FAKE, FAKE, 16, 256, 256, 254, 0, NULL, 0, NULL) == 2       # ldc < N
+
+
+def test_linear_kernel_selection(lib):
+    """Which GEMM kernel the linear entries run (a pure host function)."""
+    f = lib.w4a4_linear_kernel
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_int64] * 3
+    assert f(1, 3072, 3072) == 3          # one row: CUDA-core weight streaming
+    assert f(1, 3072, 13824) == 3
+    assert f(2, 3072, 6144) == 3          # M * K <= 12288
+    assert f(4, 12288, 3072) == 3
+    assert f(4, 5120, 5120) == 1          # more work per weight byte: split-K tensor cores
+    assert f(16, 12288, 3072) == 1
+    assert f(64, 3072, 12288) == 1
+    assert f(65, 3072, 3072) == 0         # tcgen05 GEMM
+    assert f(4608, 3072, 3072) == 0
 
 
 def test_workspace_sizes_are_host_functions(lib):

@@ -107,6 +107,29 @@ def test_gemm_smallm_exact(cuda_lib, M, N, K):
     assert np.array_equal(acc0, want)
 
 
+@pytest.mark.parametrize("M", [1, 2, 3, 4])
+@pytest.mark.parametrize("N,K", [(8, 32), (392, 3072), (3072, 12288), (1000, 24576), (12288, 3072), (4744, 256)])
+def test_gemm_tiny_m_exact(cuda_lib, M, N, K):
+    """The CUDA-core weight-streaming kernel (gemm_s32 path 3): ragged row
+    groups of 1, 2 and 4 rows per warp step, K from one 16-byte chunk per row
+    up to the largest widened activation that fits (4 x 24576 bytes)."""
+    qa, qb = _codes((M, K), 15 + M), _codes((N, K), 16 + N)
+    acc = cuda_lib.gemm_s32(_packed_cuda(qa), _packed_cuda(qb), path=3).cpu().numpy()
+    assert np.array_equal(acc, orc.gemm_s32(orc.pack_int4(qa), orc.pack_int4(qb)))
+
+
+def test_gemm_tiny_m_extremes(cuda_lib):
+    """+-7 everywhere reaches the +-49 K bound of the accumulator."""
+    K, N = 24576, 24
+    qa = np.full((4, K), 7, dtype=np.int8)
+    qa[1] = -7
+    qb = np.full((N, K), 7, dtype=np.int8)
+    qb[::2] = -7
+    acc = cuda_lib.gemm_s32(_packed_cuda(qa), _packed_cuda(qb), path=3).cpu().numpy()
+    assert np.array_equal(acc, orc.gemm_s32(orc.pack_int4(qa), orc.pack_int4(qb)))
+    assert np.abs(acc).max() == 49 * K
+
+
 def test_full_size_paths_agree(cuda_lib):
     """At the square layer's size the tensor-core kernel's accumulators equal
     an exact fp64 product on the GPU (integers below 2^53), and its bf16

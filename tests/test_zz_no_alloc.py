@@ -36,7 +36,7 @@ def _call(lib, Xq, sx, Wq, sw, b, y):
     return lib.w4a4_linear_noalloc(P(Xq), P(sx), P(Wq), P(sw), P(b), P(y), M, N, 2 * Kh, y.stride(0), stream)
 
 
-@pytest.mark.parametrize("M,N,K", [(8, 3072, 3072), (16, 392, 3072), (1, 5120, 5120), (33, 1024, 1024)])
+@pytest.mark.parametrize("M,N,K", [(8, 3072, 3072), (16, 392, 3072), (1, 5120, 5120), (33, 1024, 1024), (2, 3072, 3072), (3, 4096, 4096)])
 def test_no_alloc_matches_workspace_entry(cuda_lib, M, N, K):
     lib = cuda_lib.load_library()
     Xq, sx, Wq, sw, b = _operands(cuda_lib, M, N, K, seed=M + N)

@@ -41,6 +41,7 @@ SIGNATURES = {
     "w4a4_linear": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P, _SZ, _P]),
     "w4a4_linear_fused": (_I, [_P, _I64, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I, _I, _P, _SZ, _P]),
     "w4a4_workspace_bytes": (_SZ, [_I64, _I64, _I64]),
+    "w4a4_linear_kernel": (_I, [_I64, _I64, _I64]),
     "w4a4_fused_workspace_bytes": (_SZ, [_I64, _I64, _I64]),
     "w4a4_gemm_s32": (_I, [_P, _P, _P, _I64, _I64, _I64, _I64, _I, _P, _SZ, _P]),
     "w4a4_linear_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P]),
@@ -104,6 +105,13 @@ def _bits(t):
 # Workspaces (the fused entry's packed activation and scales) are cached per
 # (purpose, device, stream) and grown on demand.
 _workspaces = {}
+
+
+def linear_kernel(M, N, K):
+    """The GEMM kernel linear() and linear_fused() run for this shape, as
+    gemm_s32's path number (0 tcgen05 GEMM, 1 small-M split-K, 3 tiny-M
+    CUDA-core)."""
+    return int(load_library().w4a4_linear_kernel(M, N, K))
 
 
 def workspace(nbytes, device, kind="linear"):
@@ -179,7 +187,8 @@ def linear_fused(x, Wq, sw, bias=None, g=128, act=0, out=None):
 
 def gemm_s32(Xq, Wq, path=0, out=None):
     """Raw int32 accumulators acc [M, N] (path 0: tcgen05 kernel, 1: small-M
-    kernel, 2: the warp-level mma.sync comparison kernel)."""
+    kernel, 2: the warp-level mma.sync comparison kernel, 3: the tiny-M
+    CUDA-core kernel, M <= 4)."""
     lib = load_library()
     _need_cuda(Xq, torch.int8, "Xq")
     _need_cuda(Wq, torch.int8, "Wq")

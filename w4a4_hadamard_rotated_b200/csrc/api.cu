@@ -142,6 +142,15 @@ int smallm_threshold() {
   return v;
 }
 
+// The weight-streaming kernels by batch size: the CUDA-core one for a few
+// rows, the split-K tensor-core one up to smallm_threshold(), else the
+// tcgen05 GEMM.
+int linear_path(int64_t M, int64_t K) {
+  const int64_t small = smallm_threshold();
+  if (M <= small && gemv_preferred(M, K)) return 3;
+  return M <= small ? 1 : 0;
+}
+
 int check_quant_shape(int64_t K, int g) {
   if (g != 64 && g != 128 && g != 256) return W4A4_ERR_GROUP;
   if (K < 128 || K > kQuantMaxK || K % 128 != 0) return W4A4_ERR_SHAPE;
@@ -160,7 +169,8 @@ int check_gemm_shape(int64_t M, int64_t N, int64_t K) {
 
 // Shared body of w4a4_linear / w4a4_gemm_s32 after validation.  path 0: the
 // tcgen05 tensor-core kernel; 1: the small-M weight-streaming kernel; 2: the
-// warp-level mma.sync comparison kernel (int32 output only).
+// warp-level mma.sync comparison kernel (int32 output only); 3: the tiny-M
+// weight-streaming kernel on the CUDA cores.
 int run_linear(const int8_t* Xq, const float* sx, const int8_t* Wq, const float* sw, const uint16_t* bias, void* out,
                int64_t M, int64_t N, int64_t K, int64_t ldo, int out_s32, int path, cudaStream_t stream,
                int early_w = 0) {
@@ -168,6 +178,21 @@ int run_linear(const int8_t* Xq, const float* sx, const int8_t* Wq, const float*
   int st = current_device(&dev);
   if (st != W4A4_OK) return st;
   if (M == 0) return W4A4_OK;
+  if (path == 3) {
+    GemvArgs a{};
+    a.xq = Xq;
+    a.sx = sx;
+    a.wq = Wq;
+    a.sw = sw;
+    a.bias = bias;
+    a.out = out;
+    a.M = M;
+    a.N = N;
+    a.K = K;
+    a.ldo = ldo;
+    a.out_s32 = out_s32;
+    return gemv_launch(a, dev->num_sms, stream) == cudaSuccess ? W4A4_OK : W4A4_ERR_CUDA;
+  }
   if (path == 2) {
     CUtensorMap tmA, tmB;
     if ((st = packed_map(&tmA, Xq, M, K, 128, true)) != W4A4_OK) return st;
@@ -314,6 +339,11 @@ int w4a4_quantize_activation(const uint16_t* x, int64_t M, int64_t K, int64_t ld
 // No kernel of the linear needs a workspace any more (the small-M kernel
 // reduces its K slices on chip); the workspace arguments of w4a4_linear and
 // w4a4_gemm_s32 are kept for ABI stability and may be NULL.
+int w4a4_linear_kernel(int64_t M, int64_t N, int64_t K) {
+  (void)N;
+  return linear_path(M, K);
+}
+
 size_t w4a4_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   (void)M;
   (void)N;
@@ -336,7 +366,7 @@ int w4a4_linear(const int8_t* Xq, const float* sx, const int8_t* Wq, const float
                 void* stream) {
   int st = validate_linear(Xq, sx, Wq, sw, bias, y, M, N, K, ldy, 0);
   if (st != W4A4_OK) return st;
-  const int path = (M <= smallm_threshold()) ? 1 : 0;
+  const int path = linear_path(M, K);
   (void)workspace;
   (void)workspace_bytes;
   return run_linear(Xq, sx, Wq, sw, bias, y, M, N, K, ldy, 0, path, static_cast<cudaStream_t>(stream));
@@ -346,8 +376,9 @@ int w4a4_gemm_s32(const int8_t* Xq, const int8_t* Wq, int32_t* acc, int64_t M, i
                   int path, void* workspace, size_t workspace_bytes, void* stream) {
   int st = validate_linear(Xq, nullptr, Wq, nullptr, nullptr, acc, M, N, K, ldc, 1);
   if (st != W4A4_OK) return st;
-  if (path != 0 && path != 1 && path != 2) return W4A4_ERR_ARG;
+  if (path < 0 || path > 3) return W4A4_ERR_ARG;
   if (path == 1 && M > kSmallMMax) return W4A4_ERR_SHAPE;
+  if (path == 3 && M != 0 && !gemv_fits(M, K)) return W4A4_ERR_SHAPE;
   (void)workspace;
   (void)workspace_bytes;
   return run_linear(Xq, nullptr, Wq, nullptr, nullptr, acc, M, N, K, ldc, 1, path, static_cast<cudaStream_t>(stream));
@@ -379,7 +410,7 @@ int w4a4_linear_fused(const uint16_t* x, int64_t ldx, const int8_t* Wq, const fl
   float* sx = reinterpret_cast<float*>(ws + fused_codes_bytes(M, K));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if ((st = w4a4_quantize_activation(x, M, K, ldx, g, act, xq, sx, stream)) != W4A4_OK) return st;
-  const int path = (M <= smallm_threshold()) ? 1 : 0;
+  const int path = linear_path(M, K);
   // The quantiser above is launched in plain stream order, so whatever wrote
   // the weights finished before it started: the small-M kernel may begin
   // streaming them before its grid-dependency wait.

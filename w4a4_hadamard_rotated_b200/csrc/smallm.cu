@@ -514,8 +514,9 @@ int smallm_rows_padded(int64_t M) { return M <= 16 ? 16 : (M <= 32 ? 32 : 64); }
 
 // ---------------------------------------------------------------------------
 // Small-M linear that allocates nothing (w4a4_linear_noalloc in w4a4.h): the
-// small-M kernel reduces its K slices on chip, so it needs no scratch memory
-// at all; this entry takes no workspace argument.
+// small-M kernel reduces its K slices on chip and the tiny-M kernel keeps its
+// operands in one CTA, so neither needs scratch memory; this entry takes no
+// workspace argument.
 // ---------------------------------------------------------------------------
 #include "w4a4.h"
 
@@ -528,6 +529,22 @@ extern "C" int w4a4_linear_noalloc(const int8_t* Xq, const float* sx, const int8
   if (M < 1 || M > kSmallMMax) return W4A4_ERR_SHAPE;
   DeviceInfo* dev = nullptr;
   if ((st = current_device(&dev)) != W4A4_OK) return st;
+  if (gemv_preferred(M, K)) {
+    // a few rows: the CUDA-core weight-streaming kernel, which needs no scratch either
+    GemvArgs g{};
+    g.xq = Xq;
+    g.sx = sx;
+    g.wq = Wq;
+    g.sw = sw;
+    g.bias = bias;
+    g.out = y;
+    g.M = M;
+    g.N = N;
+    g.K = K;
+    g.ldo = ldy;
+    g.out_s32 = 0;
+    return gemv_launch(g, dev->num_sms, static_cast<cudaStream_t>(stream)) == cudaSuccess ? W4A4_OK : W4A4_ERR_CUDA;
+  }
   CUtensorMap tmW, tmX;
   if ((st = packed_map(&tmW, Wq, N, K, WM, true)) != W4A4_OK) return st;
   if ((st = packed_map(&tmX, Xq, M, K, smallm_rows_padded(M))) != W4A4_OK) return st;

@@ -94,4 +94,29 @@ cudaError_t smallm_launch_tm(const CUtensorMap& tmW, const CUtensorMap& tmX, con
 int smallm_rows_padded(int64_t M);
 constexpr int kSmallMMax = 64;
 
+// ---- tiny-M weight streaming on the CUDA cores (gemv.cu)
+struct GemvArgs {
+  const int8_t* xq;       // [M, K/2]
+  const float* sx;        // [M]
+  const int8_t* wq;       // [N, K/2]
+  const float* sw;        // [N]
+  const uint16_t* bias;   // [N] bf16 bits or NULL
+  void* out;              // y [M, ldo] bf16, or acc [M, ldo] int32 when out_s32
+  int64_t M, N, K, ldo;
+  int out_s32;
+};
+constexpr int kGemvMaxM = 4;
+// widened activations (M * K bytes) live in one CTA's shared memory
+constexpr size_t kGemvMaxSmem = 96 * 1024;
+inline bool gemv_fits(int64_t M, int64_t K) {
+  return M >= 1 && M <= kGemvMaxM && static_cast<size_t>(M) * static_cast<size_t>(K) <= kGemvMaxSmem;
+}
+// The shapes the linear entries route to it: measured against the split-K
+// tensor-core kernel (CUDA-graph replay, N x K in {12288 x 3072, 3072 x 12288,
+// 5120^2, 3072^2}) it is faster for every M = 1 shape (6.2 vs 10.7 us at
+// 12288 x 3072) and whenever M * K <= 12288; above that each weight byte
+// costs too many shared-memory reads of the activations.
+inline bool gemv_preferred(int64_t M, int64_t K) { return gemv_fits(M, K) && (M == 1 || M * K <= 12288); }
+cudaError_t gemv_launch(const GemvArgs& a, int num_sms, cudaStream_t stream);
+
 }  // namespace w4a4
