@@ -191,6 +191,7 @@ int run_linear(const int8_t* Xq, const float* sx, const int8_t* Wq, const float*
     a.K = K;
     a.ldo = ldo;
     a.out_s32 = out_s32;
+    a.early_w = early_w;
     return gemv_launch(a, dev->num_sms, stream) == cudaSuccess ? W4A4_OK : W4A4_ERR_CUDA;
   }
   if (path == 2) {

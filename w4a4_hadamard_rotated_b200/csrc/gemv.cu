@@ -25,6 +25,9 @@
 //     0 .. RPW*M-1 apply y = bf16(((float)acc * sx[m]) * sw[n] + bias[n]) with
 //     separately rounded fp32 steps, or store acc for the int32 entry.
 //   * Grid: warps walk row groups with a grid stride over ~2 CTAs per SM.
+//     In the fused layer each warp first requests all of its weight rows into
+//     L2 with bulk prefetches, before the grid-dependency wait, so the weight
+//     stream overlaps the activation quantiser.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -62,12 +65,29 @@ template <int M, int RPW, int OUT_S32>
 __global__ void __launch_bounds__(kGemvThreads, 2)
     gemv_kernel(const int8_t* __restrict__ xq, const float* __restrict__ sx, const int8_t* __restrict__ wq,
                 const float* __restrict__ sw, const uint16_t* __restrict__ bias, void* __restrict__ out,
-                int64_t N, int64_t K, int64_t ldo) {
+                int64_t N, int64_t K, int64_t ldo, int early_w) {
   extern __shared__ uint2 xw[];
   const int words = static_cast<int>(K / 8);   // packed 32-bit words per row
   const int chunks = words / 4;                // 16-byte chunks per row (K % 32 == 0)
-  // A grid-dependency wait first: the packed activations may come from the
-  // previous kernel of the stream (the activation quantiser of a fused layer).
+  const int lane = threadIdx.x & 31;
+  const int64_t warp_global = static_cast<int64_t>(blockIdx.x) * kGemvWarps + (threadIdx.x >> 5);
+  const int64_t warps_total = static_cast<int64_t>(gridDim.x) * kGemvWarps;
+  const int64_t groups = (N + RPW - 1) / RPW;
+  // With early_w the weights were complete before the previous kernel of the
+  // stream started (the fused entry): every weight row this warp will read is
+  // requested into L2 now (one bulk prefetch per row, spread over the lanes),
+  // so the weight stream overlaps that kernel.  (Issued after the wait, the
+  // prefetches overlap nothing and measured slower than the plain loads.)
+  if (early_w) {
+    int idx = 0;
+    for (int64_t grp = warp_global; grp < groups; grp += warps_total)
+      for (int r = 0; r < RPW; ++r, ++idx) {
+        const int64_t n = grp * RPW + r;
+        if (n < N && (idx & 31) == lane) bulk_prefetch_l2(wq + n * (K / 2), static_cast<uint32_t>(K / 2));
+      }
+  }
+  // The packed activations may come from the previous kernel of the stream
+  // (the activation quantiser of a fused layer).
   griddep_wait();
   for (int i = threadIdx.x; i < M * words; i += kGemvThreads) {
     const int m = i / words;
@@ -79,10 +99,6 @@ __global__ void __launch_bounds__(kGemvThreads, 2)
   }
   __syncthreads();
 
-  const int lane = threadIdx.x & 31;
-  const int64_t warp_global = static_cast<int64_t>(blockIdx.x) * kGemvWarps + (threadIdx.x >> 5);
-  const int64_t warps_total = static_cast<int64_t>(gridDim.x) * kGemvWarps;
-  const int64_t groups = (N + RPW - 1) / RPW;
   for (int64_t grp = warp_global; grp < groups; grp += warps_total) {
     const int64_t n0 = grp * RPW;
     int32_t acc[RPW][M];
@@ -175,7 +191,7 @@ cudaError_t launch_m(const GemvArgs& a, int num_sms, cudaStream_t stream) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   e = cudaLaunchKernelEx(&cfg, gemv_kernel<M, RPW, OUT_S32>, a.xq, a.sx, a.wq, a.sw, a.bias, a.out, a.N, a.K,
-                         a.ldo);
+                         a.ldo, a.early_w);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -104,6 +104,7 @@ struct GemvArgs {
   void* out;              // y [M, ldo] bf16, or acc [M, ldo] int32 when out_s32
   int64_t M, N, K, ldo;
   int out_s32;
+  int early_w;            // as SmallMArgs::early_w
 };
 constexpr int kGemvMaxM = 4;
 // widened activations (M * K bytes) live in one CTA's shared memory
