@@ -130,6 +130,39 @@ def test_gemm_tiny_m_extremes(cuda_lib):
     assert np.abs(acc).max() == 49 * K
 
 
+@pytest.mark.parametrize("M,K,g", [(1, 3072, 128), (1, 12288, 128), (2, 6144, 64), (3, 4096, 256),
+                                   (4, 3072, 128), (1, 256, 256), (4, 1024, 64), (2, 2048, 128)])
+def test_fused_tiny_m_matches_separate_calls(cuda_lib, M, K, g):
+    """For a few rows the fused entry (the tiny-M kernel streaming its weights
+    into L2 while the activations are quantised) gives outputs, codes and
+    scales bit-identical to the activation kernel followed by the linear
+    entry, with strided activation rows and an all-zero row."""
+    N = 1000 + 8 * M   # ragged row groups
+    cfg = workloads.Linear("tiny fused", M=M, K=K, N=N, g=g, seed=40 + M + K // 256)
+    x, W, b = cfg.make()
+    if M > 1:
+        x[1] = 0   # scale 0, codes 0, y = bias
+    wide = torch.zeros(M, K + 64, dtype=torch.bfloat16)
+    wide[:, :K] = x
+    xs = wide.cuda()[:, :K]
+    Wq, sw = cuda_lib.quantize_weight(W.cuda(), g)
+    bc = b.cuda()
+    assert cuda_lib.linear_kernel(M, N, K) == 3
+    y1 = cuda_lib.linear_fused(xs, Wq, sw, bc, g)
+    nbytes = cuda_lib.load_library().w4a4_fused_workspace_bytes(M, N, K)
+    ws = cuda_lib.workspace(nbytes, xs.device, "fused")
+    codes = ws[: M * K // 2].view(torch.int8).view(M, K // 2).clone()
+    off = (M * K // 2 + 255) // 256 * 256
+    scales = ws[off: off + 4 * M].view(torch.float32).clone()
+    Xq, sx = cuda_lib.quantize_activation(xs, g)
+    y2 = cuda_lib.linear(Xq, sx, Wq, sw, bc)
+    assert torch.equal(codes, Xq)
+    assert torch.equal(scales.view(torch.int32), sx.view(torch.int32))
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+    ref = orc.quantize_activation(workloads.bf16_bits(x), g)
+    check_packed(codes, scales, ref, f"fused tiny {M}x{K} g{g}")
+
+
 def test_full_size_paths_agree(cuda_lib):
     """At the square layer's size the tensor-core kernel's accumulators equal
     an exact fp64 product on the GPU (integers below 2^53), and its bf16
