@@ -412,9 +412,10 @@ int w4a4_linear_fused(const uint16_t* x, int64_t ldx, const int8_t* Wq, const fl
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if ((st = w4a4_quantize_activation(x, M, K, ldx, g, act, xq, sx, stream)) != W4A4_OK) return st;
   const int path = linear_path(M, K);
-  // The quantiser above is launched in plain stream order, so whatever wrote
-  // the weights finished before it started: the small-M kernel may begin
-  // streaming them before its grid-dependency wait.
+  // The quantiser above lets the next kernel start only after its own
+  // grid-dependency wait, i.e. once everything before it has finished, so
+  // whatever wrote the weights is complete when the GEMM kernel starts: the
+  // weight-streaming kernels may begin reading them before their own wait.
   return run_linear(xq, sx, Wq, sw, bias, y, M, N, K, ldy, 0, path, s, 1);
 }
 

@@ -73,8 +73,9 @@ __global__ void __launch_bounds__(kGemvThreads, 2)
   const int64_t warp_global = static_cast<int64_t>(blockIdx.x) * kGemvWarps + (threadIdx.x >> 5);
   const int64_t warps_total = static_cast<int64_t>(gridDim.x) * kGemvWarps;
   const int64_t groups = (N + RPW - 1) / RPW;
-  // With early_w the weights were complete before the previous kernel of the
-  // stream started (the fused entry): every weight row this warp will read is
+  // With early_w the weights were complete before this kernel started (the
+  // fused entry's quantiser lets it start only after its own grid-dependency
+  // wait): every weight row this warp will read is
   // requested into L2 now (one bulk prefetch per row, spread over the lanes),
   // so the weight stream overlaps that kernel.  (Issued after the wait, the
   // prefetches overlap nothing and measured slower than the plain loads.)

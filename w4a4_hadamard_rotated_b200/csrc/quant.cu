@@ -219,10 +219,8 @@ __global__ void __maxnreg__(96)
   const size_t row_bytes = static_cast<size_t>(K) * sizeof(TIn);
   const size_t stage_bytes = static_cast<size_t>(P) * row_bytes;
 
-  // every CTA of this persistent grid is resident now: the next kernel of the
-  // stream (the GEMM of a fused layer) may be scheduled as SMs free up; it
-  // waits for this grid's writes before it reads them
-  griddep_launch_dependents();
+  // Set-up that reads nothing a previous kernel may write (the GELU table is
+  // filled by a synchronous host copy before any launch that uses it).
   for (int i = tid; i < 3 * kMaxRows; i += blockDim.x) (&row_amax[0][0])[i] = 0u;
   if (ACT == 1)
     for (int i = tid; i < kGeluTableSize; i += blockDim.x) gelu_tab[i] = g_gelu_table[i];
@@ -231,6 +229,14 @@ __global__ void __maxnreg__(96)
     abort_flag = 0;
     fence_mbar_init();
   }
+  // Launched with programmatic stream serialization, so the set-up above may
+  // overlap the previous kernel; x is read and the outputs written only after
+  // that grid has finished.  Only then may the next kernel of the stream (the
+  // GEMM of a fused layer) be scheduled: it waits for this grid's writes
+  // before it reads them, and whatever ran before this kernel has finished
+  // before it starts (the fused layer's weight streaming relies on that).
+  griddep_wait();
+  griddep_launch_dependents();
   __syncthreads();
 
   // Thread 0 streams tile `tl` into ring slot `st`.
@@ -492,8 +498,18 @@ static cudaError_t launch_rq(const TIn* x, int64_t M, int K, int64_t ldx, int8_t
   auto kern = rotate_quant_pack_kernel<TIn, G, ACT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  kern<<<static_cast<unsigned>(pl.grid), pl.threads, smem, stream>>>(x, M, K, ldx, pl.P, pl.nst, out, scale,
-                                                                      status);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(pl.grid), 1, 1);
+  cfg.blockDim = dim3(static_cast<unsigned>(pl.threads), 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, x, M, K, ldx, pl.P, pl.nst, out, scale, status);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

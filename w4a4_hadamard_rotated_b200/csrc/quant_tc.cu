@@ -106,10 +106,6 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
   const int64_t ntiles = (M + P - 1) / P;
   const float norm = G == 64 ? 0.125f : 0.0883883476483184405f;   // 1/sqrt(g) in fp32
 
-  // every CTA of this grid is resident now: the next kernel of the stream
-  // (the GEMM of a fused layer) may be scheduled as SMs free up; it waits for
-  // this grid's writes before it reads them
-  griddep_launch_dependents();
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&bars.full[s], 1);
@@ -164,8 +160,11 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  // nothing below writes global memory before the previous grid has finished
+  // nothing below writes global memory before the previous grid has finished;
+  // only then may the next kernel of the stream (the GEMM of a fused layer)
+  // be scheduled -- it waits for this grid's writes before it reads them
   griddep_wait();
+  griddep_launch_dependents();
   const uint32_t tmem_base = bars.tmem_base;
   volatile int* abort_flag = &bars.abort_flag;
 

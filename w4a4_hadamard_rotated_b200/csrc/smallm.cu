@@ -188,10 +188,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     tma_prefetch_desc(&tmW);
     tma_prefetch_desc(&tmX);
     if (args.early_w) {
-      // The packed weights were written before the previous kernel of the
-      // stream started (the caller guarantees it), so their first ring
-      // stages stream in from the first cycle, before tensor memory is
-      // allocated and before the previous kernel has finished.
+      // The packed weights were complete before this kernel started (the
+      // caller guarantees it), so their first ring stages stream in from the
+      // first cycle, before tensor memory is allocated and while the
+      // previous kernel (the activation quantiser) is still running.
       const int pre = min(Lay::kSP, nkb);
       for (int i = 0; i < pre; ++i) {
         mbar_arrive_expect_tx(&bars.full[i], Lay::kPackW + Lay::kPackX);

@@ -79,10 +79,11 @@ struct SmallMArgs {
   int64_t ldo;
   int out_s32;
   unsigned int* status;   // device status word
-  // 1: the packed weights (and their scales) were complete before the
-  // previous kernel of the stream started, so the kernel may read them
-  // before its grid-dependency wait (set by the fused entry, whose previous
-  // kernel is its own activation quantiser); 0: read nothing before the wait
+  // 1: the packed weights (and their scales) were complete before this
+  // kernel started, so it may read them before its grid-dependency wait (set
+  // by the fused entry, whose previous kernel is its own activation
+  // quantiser, which lets its dependents start only after its own wait); 0:
+  // read nothing before the wait
   int early_w;
 };
 // tmW: packed weights [N, K/2] bytes, box {64, 128}, 64-byte swizzle; tmX:
