@@ -35,6 +35,8 @@ def _packed_cuda(q):
     # (whole rows per 128-lane tile: 5 x 24, 1 x 96, 3 x 40, 1 x 108, 2 x 48 lanes)
     (777, 3072, 128, 0), (520, 12288, 128, 0), (513, 5120, 128, 0), (1000, 13824, 128, 0), (600, 3072, 64, 0),
     (700, 256, 128, 0),
+    # one group per row (up to 128 rows per tile) and 128 groups per row (one row per tile)
+    (40000, 128, 128, 0), (512, 8192, 64, 0),
 ])
 def test_quantize_activation_parity(cuda_lib, M, K, g, act):
     x = workloads.make_activation(M, K, seed=M + K + g, outlier_frac=0.005, outlier_scale=30.0)

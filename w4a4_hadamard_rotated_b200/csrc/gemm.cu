@@ -481,9 +481,17 @@ int max_clusters(int num_sms) {
 template <int OUT_S32>
 cudaError_t launch(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmY, const GemmArgs& a,
                    int64_t tiles, int num_sms, cudaStream_t stream) {
-  cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<OUT_S32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(kSmemAlloc));
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!attr_set[dev]) {
+    e = cudaFuncSetAttribute(gemm_tc_kernel<OUT_S32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kSmemAlloc));
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
   const int64_t cmax = max_clusters<OUT_S32>(num_sms);
   const int grid = static_cast<int>(2 * (tiles < cmax ? tiles : cmax));
   cudaLaunchConfig_t cfg = {};

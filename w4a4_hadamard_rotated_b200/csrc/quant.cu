@@ -496,8 +496,18 @@ static cudaError_t launch_rq(const TIn* x, int64_t M, int K, int64_t ldx, int8_t
   if (pl.P < 1) return cudaErrorInvalidValue;
   const size_t smem = static_cast<size_t>(pl.nst) * pl.P * K * sizeof(TIn);
   auto kern = rotate_quant_pack_kernel<TIn, G, ACT>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  // the dynamic shared-memory limit is raised only when a launch needs more
+  // than this device has been given so far (the attribute call costs host time)
+  static size_t granted[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (smem > granted[dev]) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    granted[dev] = smem;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(pl.grid), 1, 1);
   cfg.blockDim = dim3(static_cast<unsigned>(pl.threads), 1, 1);
