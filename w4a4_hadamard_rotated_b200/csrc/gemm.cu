@@ -226,6 +226,111 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = bars.tmem_base;
   volatile int* abort_flag = &bars.abort_flag;
 
+  // The tile's column scales and bias, staged once in shared memory
+  // (double-buffered by tile) by the four epilogue warps, thread et taking
+  // columns et, et + 128.
+  auto stage_scales = [&](int t, int ab, int et) {
+    if (OUT_S32) return;
+    const int64_t nt0 = static_cast<int64_t>(t / num_m) * BN;
+#pragma unroll
+    for (int j = et; j < BN; j += 128) {
+      const int64_t n = nt0 + j;
+      epi_sw[ab][j] = n < N ? args.sw[n] : 0.0f;
+      epi_bias[ab][j] = (n < N && args.bias != nullptr) ? __uint_as_float(static_cast<uint32_t>(args.bias[n]) << 16)
+                                                        : 0.0f;
+    }
+  };
+  // 32-column chunks [c_begin, c_end) of tile t's accumulator (buffer ab) for
+  // this warp's 32 rows: y = bf16(((float)acc * sx) * sw (+ bias)) with each
+  // step rounded on its own, staged per 32 x 32 block in two alternating
+  // 2 KB boxes at `stage` (64-byte swizzle) and written by TMA stores.
+  auto drain_chunks = [&](int t, int ab, int c_begin, int c_end, uint8_t* stage) {
+    const int q = warp & 3;
+    const int mb = t % num_m, nb = t / num_m;
+    const int64_t nt0 = static_cast<int64_t>(nb) * BN;
+    const float* sws = epi_sw[ab];
+    const float* bs = epi_bias[ab];
+    const int64_t m = static_cast<int64_t>(mb) * BM + rank * HM + q * 32 + lane;
+    const bool mrow = m < M;
+    float sxm = 0.0f;
+    if (!OUT_S32 && mrow) sxm = args.sx[m];
+    const uint64_t sx2 = pk2(sxm, sxm);
+    const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + ab * BN;
+    // one chunk: its tensor-memory load (issued one chunk earlier) is waited
+    // for, the next chunk's load is issued into the other buffer so that it
+    // overlaps this chunk's math, and the chunk is converted and stored
+    auto chunk = [&](int c, uint32_t (&cur)[32], uint32_t (&nxt)[32]) {
+      tmem_wait_ld();
+      if (c + 1 < c_end) tmem_ld_32x32b_x32(tbase + (c + 1) * 32, nxt);
+      const int64_t n0 = nt0 + c * 32;
+      if (n0 >= N) return;   // warp-uniform; the tensor-memory loads above stay aligned
+      const bool full = n0 + 32 <= N;
+      if (OUT_S32) {
+        if (!mrow) return;
+        int32_t v[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = static_cast<int32_t>(cur[i]) >> 8;
+        int32_t* dst = reinterpret_cast<int32_t*>(args.out) + m * args.ldo + n0;
+        if (full) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            reinterpret_cast<int4*>(dst)[i] = make_int4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (n0 + i < N) dst[i] = v[i];
+        }
+        return;
+      }
+      uint32_t packed[16];
+      const float* swc = sws + c * 32;
+      const float* bc = bs + c * 32;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        // ((float)acc * sx) * sw (+ bias), each step rounded on its own
+        const uint64_t a2 = pk2(__int2float_rn(static_cast<int32_t>(cur[2 * i]) >> 8),
+                                __int2float_rn(static_cast<int32_t>(cur[2 * i + 1]) >> 8));
+        const float2 w2 = *reinterpret_cast<const float2*>(swc + 2 * i);
+        uint64_t y2 = mul2(mul2(a2, sx2), pk2(w2.x, w2.y));
+        if (args.bias != nullptr) {
+          const float2 b2 = *reinterpret_cast<const float2*>(bc + 2 * i);
+          y2 = add2(y2, pk2(b2.x, b2.y));
+        }
+        float y0, y1;
+        upk2(y2, y0, y1);
+        const __nv_bfloat162 h = __floats2bfloat162_rn(y0, y1);
+        packed[i] = *reinterpret_cast<const uint32_t*>(&h);
+      }
+      // stage the 32 x 32 block (row = lane, 64-byte swizzle: chunk j of
+      // row r at chunk j ^ ((r >> 1) & 3); conflict-free for this pattern)
+      uint8_t* box = stage + ((c & 1) * kStageBox);
+      // the store that last used this box (two chunks ago, possibly in the
+      // previous tile) must have finished reading it
+      if (lane == 0) bulk_wait_group_read<1>();
+      __syncwarp();
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        *reinterpret_cast<uint4*>(box + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4)) =
+            make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+      fence_async_shared();
+      __syncwarp();
+      // a box whose first row is past M stores nothing (rows past M inside
+      // a box are clipped by the tensor map)
+      if (lane == 0 && m < M) {
+        tma_store_2d(&tmY, box, static_cast<int32_t>(n0), static_cast<int32_t>(m));
+        bulk_commit_group();
+      }
+    };
+    // chunk ranges start on an even chunk and hold an even number of them:
+    // even chunks use buffer r0, odd ones r1 (static register indexing)
+    uint32_t r0[32], r1[32];
+    tmem_ld_32x32b_x32(tbase + c_begin * 32, r0);
+    for (int c = c_begin; c < c_end; c += 2) {
+      chunk(c, r0, r1);
+      chunk(c + 1, r1, r0);
+    }
+  };
+
   if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
     if (rank == 0 && lane == 0) {
@@ -333,26 +438,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (is_epi_warp(warp)) {
     // ------------------------------------------------------------ epilogue warps
+    // every tile but the cluster's last (drained by all sixteen warps below)
     const int q = warp & 3;   // TMEM lane quarter this warp may access
     const int et = q * 32 + lane;   // 0..127 across the four epilogue warps
     uint8_t* epi_stage = smem + kOffEpi + q * 2 * kStageBox;
     uint32_t acc_ph = 0;
     int lt = 0;
-    for (int t = cluster; t < tiles; t += nclusters, ++lt) {
+    for (int t = cluster; t + nclusters < tiles; t += nclusters, ++lt) {
       const int ab = lt & 1;
-      const int mb = t % num_m, nb = t / num_m;
-      const int64_t nt0 = static_cast<int64_t>(nb) * BN;
-      // the tile's column scales and bias, staged once (double-buffered by tile)
-      float* sws = epi_sw[ab];
-      float* bs = epi_bias[ab];
-      if (!OUT_S32) {
-#pragma unroll
-        for (int j = et; j < BN; j += 128) {
-          const int64_t n = nt0 + j;
-          sws[j] = n < N ? args.sw[n] : 0.0f;
-          bs[j] = (n < N && args.bias != nullptr) ? __uint_as_float(static_cast<uint32_t>(args.bias[n]) << 16) : 0.0f;
-        }
-      }
+      stage_scales(t, ab, et);
       (void)warp_wait_cluster(&bars.acc_full[ab], (acc_ph >> ab) & 1, abort_flag, args.status);
       acc_ph ^= 1u << ab;
       // staged scales visible to the four warps; every wait above is bounded, so
@@ -360,84 +454,36 @@ __global__ void __launch_bounds__(kThreads, 1)
       asm volatile("bar.sync 1, 128;" ::: "memory");
       if (*abort_flag) break;
       tc_fence_after();
-      const int64_t m = static_cast<int64_t>(mb) * BM + rank * HM + q * 32 + lane;
-      const bool mrow = m < M;
-      float sxm = 0.0f;
-      if (!OUT_S32 && mrow) sxm = args.sx[m];
-      const uint64_t sx2 = pk2(sxm, sxm);
-      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + ab * BN;
-      uint32_t r[2][32];
-      tmem_ld_32x32b_x32(tbase, r[0]);
-#pragma unroll
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t (&cur)[32] = r[c & 1];
-        tmem_wait_ld();
-        // the next chunk's tensor-memory load overlaps this chunk's math
-        if (c + 1 < BN / 32) tmem_ld_32x32b_x32(tbase + (c + 1) * 32, r[(c + 1) & 1]);
-        const int64_t n0 = nt0 + c * 32;
-        if (n0 >= N) continue;   // warp-uniform; the tensor-memory loads above stay aligned
-        const bool full = n0 + 32 <= N;
-        if (OUT_S32) {
-          if (!mrow) continue;
-          int32_t v[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = static_cast<int32_t>(cur[i]) >> 8;
-          int32_t* dst = reinterpret_cast<int32_t*>(args.out) + m * args.ldo + n0;
-          if (full) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-              reinterpret_cast<int4*>(dst)[i] = make_int4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-          } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (n0 + i < N) dst[i] = v[i];
-          }
-        } else {
-          uint32_t packed[16];
-          const float* swc = sws + c * 32;
-          const float* bc = bs + c * 32;
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            // ((float)acc * sx) * sw (+ bias), each step rounded on its own
-            const uint64_t a2 = pk2(__int2float_rn(static_cast<int32_t>(cur[2 * i]) >> 8),
-                                    __int2float_rn(static_cast<int32_t>(cur[2 * i + 1]) >> 8));
-            const float2 w2 = *reinterpret_cast<const float2*>(swc + 2 * i);
-            uint64_t y2 = mul2(mul2(a2, sx2), pk2(w2.x, w2.y));
-            if (args.bias != nullptr) {
-              const float2 b2 = *reinterpret_cast<const float2*>(bc + 2 * i);
-              y2 = add2(y2, pk2(b2.x, b2.y));
-            }
-            float y0, y1;
-            upk2(y2, y0, y1);
-            const __nv_bfloat162 h = __floats2bfloat162_rn(y0, y1);
-            packed[i] = *reinterpret_cast<const uint32_t*>(&h);
-          }
-          // stage the 32 x 32 block (row = lane, 64-byte swizzle: chunk j of
-          // row r at chunk j ^ ((r >> 1) & 3); conflict-free for this pattern)
-          uint8_t* box = epi_stage + ((c & 1) * kStageBox);
-          // the store that last used this box (two chunks ago, possibly in the
-          // previous tile) must have finished reading it
-          if (lane == 0) bulk_wait_group_read<1>();
-          __syncwarp();
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            *reinterpret_cast<uint4*>(box + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4)) =
-                make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
-          fence_async_shared();
-          __syncwarp();
-          // a box whose first row is past M stores nothing (rows past M inside
-          // a box are clipped by the tensor map)
-          if (lane == 0 && m < M) {
-            tma_store_2d(&tmY, box, static_cast<int32_t>(n0), static_cast<int32_t>(m));
-            bulk_commit_group();
-          }
-        }
-      }
+      drain_chunks(t, ab, 0, BN / 32, epi_stage);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_remote_smem(&bars.acc_empty[ab], 0);
     }
-    if (lane == 0) bulk_wait_group<0>();   // every store of y has completed
+  }
+
+  // ---- the cluster's last tile, drained by all sixteen warps: nothing else
+  // overlaps this epilogue, so each of the four warps of a tensor-memory lane
+  // quarter (warp % 4) takes two of the eight 32-column chunks, staging its
+  // boxes in the widened ring (idle once the last accumulator is complete).
+  // Every warp reaches the barrier below exactly once, also after an abort.
+  __syncwarp();
+  {
+    const int lt_last = (tiles - cluster + nclusters - 1) / nclusters - 1;
+    const int t_last = cluster + lt_last * nclusters;
+    const int ab = lt_last & 1;
+    if (is_epi_warp(warp)) {
+      stage_scales(t_last, ab, (warp & 3) * 32 + lane);
+      // the last accumulator's phase: uses of buffer ab before it, mod 2
+      (void)warp_wait_cluster(&bars.acc_full[ab], static_cast<uint32_t>((lt_last >> 1) & 1), abort_flag,
+                              args.status);
+    }
+    asm volatile("bar.sync 2, 512;" ::: "memory");
+    if (*abort_flag == 0) {
+      tc_fence_after();
+      const int part = warp >> 2;   // 0..3 within the lane quarter
+      drain_chunks(t_last, ab, 2 * part, 2 * part + 2, smem + warp * 2 * kStageBox);
+    }
+    if (lane == 0) bulk_wait_group_read<0>();   // every store has read its staging box
   }
 
   tc_fence_before();
