@@ -58,7 +58,9 @@ namespace w4a4 {
 
 // GELU table: Phi(t), the standard normal CDF, for the bf16 values t with
 // exponent field kGeluFirstExp .. kGeluFirstExp + kGeluExps - 1
-// (2^-12 <= |t| < 8), 128 mantissas each, positive then negative.
+// (2^-12 <= |t| < 8), 128 mantissas each; entry 2 d + sign holds the value
+// whose magnitude is the d-th of that range (the two signs side by side, so
+// the sign bit lands in the byte offset with one shift and mask).
 constexpr uint32_t kGeluFirstExp = 115;
 constexpr uint32_t kGeluExps = 15;
 constexpr int kGeluHalf = static_cast<int>(kGeluExps * 128);
@@ -106,8 +108,10 @@ __device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
 
 // GELU of the two bf16 inputs held in one 32-bit word: GELU(t) = t Phi(t)
 // with Phi(t) = (1 + erf(t / sqrt 2)) / 2 read from the table (one product,
-// so within about an ulp of the exact value).  The index is formed for both
-// halves at once with 16-bit SIMD min/max; clamping the exponent field to the
+// so within about an ulp of the exact value).  The byte offsets of both
+// entries are formed at once, one per 16-bit half (at most 8 * 1919 + 4, so
+// no half overflows): the magnitude clamped with 16-bit SIMD min/max, minus
+// the range start, times 8, plus 4 for a negative t; clamping the exponent field to the
 // table's range is the only special case: below 2^-12 the entry of 2^-12
 // stands in (Phi differs by < 1e-4, the product by < 3e-8 absolute), at or
 // above 8 the entry of 8 - 2^-4 does (Phi rounds to 1, and t Phi(t) for
@@ -117,10 +121,10 @@ __device__ __forceinline__ void gelu_phi_word(uint32_t w, const float* __restric
   uint32_t c;
   asm("max.u16x2 %0, %1, %2;" : "=r"(c) : "r"(w & 0x7FFF7FFFu), "r"(lo * 0x10001u));
   asm("min.u16x2 %0, %0, %1;" : "+r"(c) : "r"(hi * 0x10001u));
-  // entry of each half: (c - lo) + sign * kGeluHalf; no half overflows 16 bits
-  const uint32_t idx = c - lo * 0x10001u + ((w >> 15) & 0x00010001u) * static_cast<uint32_t>(kGeluHalf);
-  phi0 = tab[idx & 0xFFFFu];
-  phi1 = tab[idx >> 16];
+  const uint32_t off = ((c - lo * 0x10001u) << 3) | ((w >> 13) & 0x00040004u);
+  const char* tb = reinterpret_cast<const char*>(tab);
+  phi0 = *reinterpret_cast<const float*>(tb + (off & 0xFFFFu));
+  phi1 = *reinterpret_cast<const float*>(tb + (off >> 16));
 }
 
 // bf16 bits of element e of a 16-byte chunk.
@@ -416,7 +420,7 @@ static cudaError_t ensure_gelu_table() {
         float tf;
         std::memcpy(&tf, &fb, sizeof(tf));
         const double t = static_cast<double>(tf);
-        host[sgn * kGeluHalf + ex * 128 + f] = static_cast<float>(0.5 * (1.0 + std::erf(t / std::sqrt(2.0))));
+        host[2 * (ex * 128 + f) + sgn] = static_cast<float>(0.5 * (1.0 + std::erf(t / std::sqrt(2.0))));
       }
   e = cudaMemcpyToSymbol(g_gelu_table, host, sizeof(host));
   if (e != cudaSuccess) return e;
