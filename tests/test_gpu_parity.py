@@ -73,6 +73,49 @@ def test_quantize_zero_rows(cuda_lib):
     check_packed(Xq, sx, orc.quantize_activation(workloads.bf16_bits(x), 128), "zero rows")
 
 
+def _one_hot_rows(t_bits, K=128):
+    """Rows of K bf16 elements whose only nonzero is t in column 0 (bits)."""
+    xb = np.zeros((t_bits.size, K), dtype=np.uint16)
+    xb[:, 0] = t_bits
+    return xb
+
+
+def test_gelu_every_finite_bf16_input(cuda_lib):
+    """Every finite bf16 value t, alone in a 128-element row (g = 64, GELU on).
+    The first group rotates to GELU(t)/8 in every position and the second to
+    zeros, so the row scale sx = fl(fl(|GELU(t)| / 8) / 7) exposes the GELU
+    of each input; every code of the first group is 7 times the sign of
+    GELU(t) (0 where it is zero), every other code 0.  This reaches every
+    entry of the device's Phi table and both clamped ends (|t| < 2^-12 and
+    |t| >= 8, up to the largest bf16 values of either sign)."""
+    bits = np.arange(65536, dtype=np.uint32)
+    t_bits = bits[((bits >> 7) & 0xFF) != 0xFF].astype(np.uint16)   # Inf and NaN left out
+    xb = _one_hot_rows(t_bits)
+    x = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16)
+    Xq, sx = cuda_lib.quantize_activation(x.cuda(), 64, 1)
+    ref = orc.quantize_activation(xb, 64, 1)
+    sx_g = sx.cpu().numpy().astype(np.float64)
+    sx_r = ref["scale"].astype(np.float64)
+    # The device forms fl(t * fl(Phi(t))) against the oracle's correctly
+    # rounded GELU (about an ulp apart); below |t| = 2^-12 the entry of 2^-12
+    # stands in (< 3e-8 absolute on GELU, < 6e-10 on sx); where 1 + erf
+    # cancels in double precision (t < -5.6) both sides are below 1e-14.
+    tol = 4.0 * 2.0 ** -24 * sx_r + 6e-10
+    bad = np.flatnonzero(np.abs(sx_g - sx_r) > tol)
+    assert bad.size == 0, (f"{bad.size} inputs off, first t bits {t_bits[bad[:5]].tolist()}: "
+                           f"sx {sx_g[bad[:5]].tolist()} vs {sx_r[bad[:5]].tolist()}")
+    # the clamped top: GELU(t) = t for t >= 8 and -0 for t <= -8
+    big = ((t_bits.astype(np.uint32) >> 7) & 0xFF) >= 130
+    neg = (t_bits >> 15) == 1
+    assert np.all(sx_g[big & neg] == 0.0)
+    assert np.all(sx_g[big & ~neg] == sx_r[big & ~neg])
+    # codes: 7 times the sign wherever the oracle's GELU is clearly nonzero
+    q_g = orc.unpack_int4(Xq.cpu().numpy())
+    clear = sx_r > 1e-12
+    assert np.array_equal(q_g[clear], ref["q"][clear])
+    assert np.all(q_g[sx_g == 0] == 0)
+
+
 # --------------------------------------------------------------------------
 # K2 / K3: integer GEMM, bit-exact
 # --------------------------------------------------------------------------

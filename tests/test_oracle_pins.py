@@ -296,6 +296,16 @@ def test_gelu_matches_math_erf_and_torch():
     assert np.array_equal(got, t)
 
 
+def test_gelu_saturates_at_both_ends():
+    """GELU(t) = t Phi(t): for large positive t Phi rounds to 1 and the value
+    is t itself; for large negative t it underflows to -0, up to the largest
+    bf16 magnitudes (3.39e38)."""
+    pos = np.array([16.0, 1e3, 1e30, 3.3895e38], dtype=np.float32)
+    assert np.array_equal(orc.gelu_f32(pos), pos)
+    neg = orc.gelu_f32(-pos)
+    assert np.all(neg == 0.0) and np.all(np.signbit(neg))
+
+
 # --------------------------------------------------------------------------
 # The whole layer
 # --------------------------------------------------------------------------

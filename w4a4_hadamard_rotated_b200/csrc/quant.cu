@@ -114,8 +114,10 @@ __device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
 // the range start, times 8, plus 4 for a negative t; clamping the exponent field to the
 // table's range is the only special case: below 2^-12 the entry of 2^-12
 // stands in (Phi differs by < 1e-4, the product by < 3e-8 absolute), at or
-// above 8 the entry of 8 - 2^-4 does (Phi rounds to 1, and t Phi(t) for
-// t <= -8 is below 6e-16 |t|).  `tab` is the table in shared memory.
+// above 8 the entry of 8 - 2^-5 does, which holds 1 for positive t (Phi
+// rounds to 1 there) and 0 for negative t, so GELU is t or -0 (the exact
+// |t Phi(t)| is below 7e-15 for t <= -8 + 2^-5 and falls with |t|).  `tab`
+// is the table in shared memory.
 __device__ __forceinline__ void gelu_phi_word(uint32_t w, const float* __restrict__ tab, float& phi0, float& phi1) {
   constexpr uint32_t lo = kGeluFirstExp << 7, hi = ((kGeluFirstExp + kGeluExps) << 7) - 1u;
   uint32_t c;
@@ -400,8 +402,9 @@ __global__ void __maxnreg__(96)
 
 // Fills the GELU table of the current device once: every bf16 t with
 // 2^-12 <= |t| < 8 gets fp32(Phi(t)) = fp32((1 + erf(t / sqrt 2)) / 2)
-// evaluated in double precision.  The copy is synchronous, so the first GELU call on a
-// device must not be inside a stream capture.
+// evaluated in double precision, except t = -(8 - 2^-5), whose entry also
+// serves every t <= -8 and holds 0.  The copy is synchronous, so the first
+// GELU call on a device must not be inside a stream capture.
 static cudaError_t ensure_gelu_table() {
   static bool ready[64] = {};
   static std::mutex mu;
@@ -422,6 +425,7 @@ static cudaError_t ensure_gelu_table() {
         const double t = static_cast<double>(tf);
         host[2 * (ex * 128 + f) + sgn] = static_cast<float>(0.5 * (1.0 + std::erf(t / std::sqrt(2.0))));
       }
+  host[2 * (kGeluHalf - 1) + 1] = 0.0f;   // the clamped negative end: GELU(t <= -8) = -0
   e = cudaMemcpyToSymbol(g_gelu_table, host, sizeof(host));
   if (e != cudaSuccess) return e;
   ready[dev] = true;
