@@ -63,8 +63,8 @@ namespace w4a4 {
 // the sign bit lands in the byte offset with one shift and mask).
 constexpr uint32_t kGeluFirstExp = 115;
 constexpr uint32_t kGeluExps = 15;
-constexpr int kGeluHalf = static_cast<int>(kGeluExps * 128);
-constexpr int kGeluTableSize = 2 * kGeluHalf;
+constexpr int kGeluMags = static_cast<int>(kGeluExps * 128);   // magnitudes per sign
+constexpr int kGeluTableSize = 2 * kGeluMags;
 __device__ float g_gelu_table[kGeluTableSize];
 
 constexpr int kSlab = 64;      // elements per thread
@@ -425,7 +425,7 @@ static cudaError_t ensure_gelu_table() {
         const double t = static_cast<double>(tf);
         host[2 * (ex * 128 + f) + sgn] = static_cast<float>(0.5 * (1.0 + std::erf(t / std::sqrt(2.0))));
       }
-  host[2 * (kGeluHalf - 1) + 1] = 0.0f;   // the clamped negative end: GELU(t <= -8) = -0
+  host[2 * (kGeluMags - 1) + 1] = 0.0f;   // the clamped negative end: GELU(t <= -8) = -0
   e = cudaMemcpyToSymbol(g_gelu_table, host, sizeof(host));
   if (e != cudaSuccess) return e;
   ready[dev] = true;
