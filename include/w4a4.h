@@ -70,9 +70,9 @@ int w4a4_version(void);
 
 /*
  * Offline weight preparation: rotate (ConvRot) and quantise the rows of an
- * fp32 weight.  Page "[PR #63] ...", Description: weights are "packed signed
- * int4 pairs (low-nibble-first, [N, K/2] int8 container) with fp32 [N, 1]
- * per-row scales".
+ * fp32 weight.  Page "[PR #63] ...", Description: the weight is stored as
+ * two signed 4-bit codes per byte, the even element in the low nibble, in an
+ * int8 array of N rows by K/2 bytes, with one fp32 scale per output row.
  *   W   [N, K] fp32, row stride ldw >= K (elements), 16-byte aligned, ldw % 4 == 0
  *   N >= 1;  K % 128 == 0, K % g == 0, 128 <= K <= 24576;  g in {64,128,256}
  *   Wq  [N, K/2] int8 output, contiguous rows, 16-byte aligned
@@ -99,8 +99,8 @@ int w4a4_quantize_activation(const uint16_t* x, int64_t M, int64_t K, int64_t ld
 
 /*
  * W4A4 linear on already-quantised operands: the s4 x s4 GEMM with int32
- * accumulation and the rank-one epilogue of the page's Description
- * ("per-row/per-col scales factor out of the K loop").
+ * accumulation and the rank-one epilogue of the page's Description (the row
+ * and column scales are applied once per output, after the K loop).
  *   Xq [M, K/2] int8, sx [M] fp32 (from w4a4_quantize_activation)
  *   Wq [N, K/2] int8, sw [N] fp32 (from w4a4_quantize_weight)
  *   bias [N] bf16 bits or NULL

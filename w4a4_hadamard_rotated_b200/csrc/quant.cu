@@ -1,7 +1,8 @@
 // Fused ConvRot rotate + per-row int4 quantise + pack (the activation kernel
 // of page "[PR #63] int4_tensorwise: W4A4 layout (+ConvRot) with fused CUDA
-// kernels", Description: "FHT rotation ... + rowwise int4 quantize + pack in
-// one pass").  The same kernel, with fp32 input, prepares the weights offline.
+// kernels", Description: the rotation, the per-row quantisation and the
+// packing happen in a single kernel pass over the activations).  The same
+// kernel, with fp32 input, prepares the weights offline.
 //
 // B200 design (an HBM-bound pass that is close to ALU-bound as well: 2 bytes
 // read, half a byte written, ~log2(g) adds per code)
