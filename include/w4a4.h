@@ -82,8 +82,9 @@ int w4a4_quantize_weight(const float* W, int64_t N, int64_t K, int64_t ldw, int 
                          int8_t* Wq, float* sw, void* stream);
 
 /*
- * Run-time activation preparation (the fused "FHT rotation + rowwise int4
- * quantize + pack in one pass" kernel of the page's Description).
+ * Run-time activation preparation: the page's Description fuses the
+ * Hadamard rotation, the per-row int4 quantisation and the packing into one
+ * kernel, and so does this call.
  *   x   [M, K] bf16 bits, row stride ldx >= K, 16-byte aligned, ldx % 8 == 0
  *   act 0: none; 1: exact-erf GELU applied to x before the rotation (used to
  *       feed an MLP down projection from the up projection's output).  The

@@ -1,10 +1,10 @@
 // s4 x s4 -> s32 GEMM with the rank-one epilogue, on the sm_100a tensor cores.
 //
 // The page "[PR #63] int4_tensorwise: W4A4 layout (+ConvRot) with fused CUDA
-// kernels" (Description) keeps the per-row and per-column scales out of the K
-// loop, so the main loop is a pure integer product with int32 accumulators
-// (|acc| <= 49*K) and y = acc * sx[m] * sw[n] (+ bias) is applied once per
-// output.  Its kernel is an Ampere/Ada mma.sync s4 design; on sm_100a there is
+// kernels" (Description) applies the row and column scales only after the
+// reduction over K: the inner loop multiplies integer codes into int32
+// accumulators (|acc| <= 49*K), and y = acc * sx[m] * sw[n] (+ bias) is
+// formed once per output.  Its kernel is an Ampere/Ada mma.sync s4 design; on sm_100a there is
 // no 4-bit integer tcgen05 kind, so this kernel widens the packed nibbles to
 // bytes in shared memory and runs tcgen05.mma.kind::i8.
 //
