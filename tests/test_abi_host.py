@@ -134,3 +134,47 @@ def test_workspace_sizes_are_host_functions(lib):
 def test_debug_timeout_rejects_bad_limit(lib):
     assert lib.w4a4_debug_wait_timeout(0, NULL) == 9
     assert lib.w4a4_debug_wait_timeout(10_000_000, NULL) == 9
+
+
+def test_binding_refuses_host_tensors():
+    """No host fallback: every compute call of the binding rejects tensors
+    that are not on a CUDA device before calling the library."""
+    import torch
+    x = torch.zeros(4, 128, dtype=torch.bfloat16)
+    W = torch.zeros(8, 128, dtype=torch.float32)
+    q = torch.zeros(4, 64, dtype=torch.int8)
+    qw = torch.zeros(8, 64, dtype=torch.int8)
+    s4, s8 = torch.ones(4), torch.ones(8)
+    calls = [
+        lambda: w4.quantize_weight(W),
+        lambda: w4.quantize_activation(x),
+        lambda: w4.linear(q, s4, qw, s8),
+        lambda: w4.linear_fused(x, qw, s8),
+        lambda: w4.gemm_s32(q, qw),
+        lambda: w4.linear_noalloc(q, s4, qw, s8),
+    ]
+    for call in calls:
+        with pytest.raises(TypeError, match="CUDA tensor"):
+            call()
+
+
+def test_missing_library_fails_loudly():
+    saved = w4._lib
+    try:
+        w4._lib = None
+        with pytest.raises(RuntimeError, match="missing"):
+            w4.load_library(os.path.join(ROOT, "no_such_dir", "libw4a4.so"))
+    finally:
+        w4._lib = saved
+
+
+def test_product_code_never_touches_the_oracle():
+    """The package and the C++/CUDA sources neither import nor name the
+    oracle (it is test infrastructure only)."""
+    pkg = os.path.join(ROOT, "w4a4_hadamard_rotated_b200")
+    for dirpath, _, names in os.walk(pkg):
+        for n in names:
+            if n.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                text = open(os.path.join(dirpath, n)).read()
+                assert not re.search(r"^\s*(import|from)\s+oracle\b", text, flags=re.M), n
+                assert "w4a4_oracle" not in text, n
