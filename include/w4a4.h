@@ -135,9 +135,8 @@ int w4a4_linear_fused(const uint16_t* x, int64_t ldx, const int8_t* Wq, const fl
 
 /* Which GEMM kernel w4a4_linear and w4a4_linear_fused run for this shape,
  * numbered as w4a4_gemm_s32's path: 0 = tcgen05 tensor-core kernel, 1 =
- * small-M split-K kernel, 3 = tiny-M CUDA-core kernel.  (w4a4_linear_noalloc,
- * for M <= 64, runs 3 where this returns 3 and 1 otherwise.)  Pure host
- * function; it reads the environment switches above. */
+ * small-M split-K kernel, 3 = tiny-M CUDA-core kernel.  Pure host function;
+ * it reads the environment switches above. */
 int w4a4_linear_kernel(int64_t M, int64_t N, int64_t K);
 
 /* Workspace sizes in bytes (0 when none is needed: w4a4_workspace_bytes is
@@ -161,25 +160,36 @@ int w4a4_gemm_s32(const int8_t* Xq, const int8_t* Wq, int32_t* acc, int64_t M, i
                   void* stream);
 
 /*
- * Small-M W4A4 linear (1 <= M <= 64) that allocates nothing and takes no
- * workspace.  The pages have no counterpart to this entry point; it exists
- * for callers that cannot allocate device memory when they run the layer --
- * for instance a plug-in whose host framework owns every byte of device
- * memory and hands a custom op no scratch, or a latency-critical decode loop
- * that must not call cudaMalloc after start-up (an allocation can
- * synchronise the device and fragment a pool sized in advance).
- *   Arguments, layouts and results are those of w4a4_linear; the output is
- *   bit-identical to it.  The small-M kernel reduces its K slices in the
- *   shared memory of a CTA cluster, and the tiny-M kernel (M <= 4) keeps its
- *   operands in one CTA's registers and shared memory, so no scratch memory
- *   of any kind is used: neither a caller workspace nor memory of the
- *   library's own.
- *   M > 64 gives W4A4_ERR_SHAPE before anything is launched.  Calls are
- *   independent (they may overlap on the GPU).
+ * The fused layer of w4a4_linear_fused for callers that cannot allocate
+ * device memory.  The pages have no counterpart to this entry point.  The
+ * fused layer needs scratch memory between its two kernels (the packed
+ * activation and its row scales); w4a4_linear_fused takes it from the
+ * caller as a workspace, but some callers cannot provide one: a plug-in
+ * whose host framework owns every byte of device memory and hands a custom
+ * op only its inputs and outputs, or a serving loop that must not call
+ * cudaMalloc once it runs (an allocation can synchronise the device and
+ * fragment a pool sized in advance).  This entry point keeps that scratch in
+ * a fixed 8 MiB array inside the library instead, and neither allocates nor
+ * frees anything.
+ *   Arguments, layouts and results are those of w4a4_linear_fused without
+ *   the workspace; the output is bit-identical to it.
+ *   Size limit: the scratch must hold round256(M * K / 2) + round256(4 * M)
+ *   bytes (w4a4_fused_workspace_bytes), at most 8 MiB -- e.g. M = 4608 at
+ *   K = 3072, or any M <= 64 at K <= 32768.  Larger shapes return
+ *   W4A4_ERR_SHAPE before anything is launched.
+ *   The array exists once per GPU on which the library is loaded and holds
+ *   its 8 MiB until the process exits.  The first call on a device looks up
+ *   the array's device address (a CUDA runtime query, no allocation); make
+ *   that first call before any stream capture.
+ *   Every call on a device shares the one array, and it keeps the last
+ *   call's contents (nothing needs to start at zero: the activation kernel
+ *   writes all of it before the GEMM reads it).  Calls that overlap on the
+ *   GPU -- on different streams, or from different host threads -- race on
+ *   the array and give wrong results: order them on one stream.
  */
-int w4a4_linear_noalloc(const int8_t* Xq, const float* sx, const int8_t* Wq, const float* sw,
-                        const uint16_t* bias, uint16_t* y, int64_t M, int64_t N, int64_t K, int64_t ldy,
-                        void* stream);
+int w4a4_linear_fused_noalloc(const uint16_t* x, int64_t ldx, const int8_t* Wq, const float* sw,
+                              const uint16_t* bias, uint16_t* y, int64_t ldy, int64_t M, int64_t N, int64_t K,
+                              int g, int act, void* stream);
 
 /*
  * Synchronise `stream`, then read and clear the device status word that

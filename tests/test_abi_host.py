@@ -151,7 +151,7 @@ def test_binding_refuses_host_tensors():
         lambda: w4.linear(q, s4, qw, s8),
         lambda: w4.linear_fused(x, qw, s8),
         lambda: w4.gemm_s32(q, qw),
-        lambda: w4.linear_noalloc(q, s4, qw, s8),
+        lambda: w4.linear_fused_noalloc(x, qw, s8),
     ]
     for call in calls:
         with pytest.raises(TypeError, match="CUDA tensor"):
@@ -178,3 +178,23 @@ def test_product_code_never_touches_the_oracle():
                 text = open(os.path.join(dirpath, n)).read()
                 assert not re.search(r"^\s*(import|from)\s+oracle\b", text, flags=re.M), n
                 assert "w4a4_oracle" not in text, n
+
+
+def test_fused_noalloc_rejects_bad_arguments_and_oversized_shapes(lib):
+    """The fused entry without a workspace checks its arguments like the fused
+    entry, and refuses shapes whose packed activation and scales do not fit
+    its fixed 8 MiB scratch, all before any CUDA call."""
+    f = lib.w4a4_linear_fused_noalloc
+    base = dict(x=FAKE, ldx=3072, wq=FAKE, sw=FAKE, bias=NULL, y=FAKE, ldy=3072, M=4608, N=3072, K=3072,
+                g=128, act=0, st=NULL)
+    call = lambda **kw: f(*({**base, **kw}).values())
+    assert call(x=NULL) == 1
+    assert call(wq=NULL) == 1
+    assert call(g=32) == 3
+    assert call(act=5) == 9
+    assert call(ldx=250) == 2
+    assert call(y=MISALIGNED) == 4
+    # round256(M * K/2) + round256(4 M) <= 8 MiB: at K = 3072 that is M <= 5447
+    assert call(M=5448) == 2
+    assert call(M=4608, K=12288, ldx=12288) == 2
+    assert call(M=32760, K=5120, ldx=5120, N=5120, ldy=5120) == 2

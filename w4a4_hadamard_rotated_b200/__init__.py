@@ -44,7 +44,7 @@ SIGNATURES = {
     "w4a4_linear_kernel": (_I, [_I64, _I64, _I64]),
     "w4a4_fused_workspace_bytes": (_SZ, [_I64, _I64, _I64]),
     "w4a4_gemm_s32": (_I, [_P, _P, _P, _I64, _I64, _I64, _I64, _I, _P, _SZ, _P]),
-    "w4a4_linear_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P]),
+    "w4a4_linear_fused_noalloc": (_I, [_P, _I64, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I, _I, _P]),
 
     "w4a4_last_device_error": (_I, [_P]),
     "w4a4_debug_wait_timeout": (_I, [_I64, _P]),
@@ -201,17 +201,17 @@ def gemm_s32(Xq, Wq, path=0, out=None):
     return acc
 
 
-def linear_noalloc(Xq, sx, Wq, sw, bias=None, out=None):
-    """Small-M (M <= 64) linear that takes no workspace and uses no scratch
-    memory (see w4a4_linear_noalloc in the header)."""
+def linear_fused_noalloc(x, Wq, sw, bias=None, g=128, act=0, out=None):
+    """The fused layer without a workspace: its scratch is a fixed 8 MiB array
+    inside the library (see w4a4_linear_fused_noalloc in the header; calls
+    that overlap on the GPU race on it)."""
     lib = load_library()
-    _need_cuda(Xq, torch.int8, "Xq")
-    _need_cuda(Wq, torch.int8, "Wq")
-    M, Kh = Xq.shape
+    _need_cuda(x, torch.bfloat16, "x")
+    M, K = x.shape
     N = Wq.shape[0]
-    y = out if out is not None else torch.empty(M, N, dtype=torch.bfloat16, device=Xq.device)
-    _check(lib.w4a4_linear_noalloc(_ptr(Xq), _ptr(sx), _ptr(Wq), _ptr(sw), _ptr(bias), _ptr(y), M, N, 2 * Kh,
-                                   y.stride(0), _stream(Xq)), "w4a4_linear_noalloc")
+    y = out if out is not None else torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
+    _check(lib.w4a4_linear_fused_noalloc(_ptr(x), x.stride(0), _ptr(Wq), _ptr(sw), _ptr(bias), _ptr(y), y.stride(0),
+                                         M, N, K, g, act, _stream(x)), "w4a4_linear_fused_noalloc")
     return y
 
 

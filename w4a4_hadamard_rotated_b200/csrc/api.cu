@@ -277,6 +277,22 @@ int validate_linear(const int8_t* Xq, const float* sx, const int8_t* Wq, const f
   return W4A4_OK;
 }
 
+int validate_fused(const uint16_t* x, int64_t ldx, const int8_t* Wq, const float* sw, const uint16_t* bias,
+                   const uint16_t* y, int64_t ldy, int64_t M, int64_t N, int64_t K, int g, int act) {
+  if (Wq == nullptr || sw == nullptr) return W4A4_ERR_NULL;
+  // an empty batch (M == 0) may pass NULL for its zero-size tensors
+  if (M != 0 && (x == nullptr || y == nullptr)) return W4A4_ERR_NULL;
+  int st = check_quant_shape(K, g);
+  if (st != W4A4_OK) return st;
+  if (act != 0 && act != 1) return W4A4_ERR_ARG;
+  if ((st = check_gemm_shape(M, N, K)) != W4A4_OK) return st;
+  if (ldx < K || ldy < N) return W4A4_ERR_SHAPE;
+  if (ldx % 8 != 0 || !aligned(x, 16)) return W4A4_ERR_ALIGN;
+  if (ldy % 8 != 0 || !aligned(y, 16) || !aligned(Wq, 16) || !aligned(sw, 16)) return W4A4_ERR_ALIGN;
+  if (bias != nullptr && !aligned(bias, 16)) return W4A4_ERR_ALIGN;
+  return W4A4_OK;
+}
+
 }  // namespace w4a4
 
 using namespace w4a4;
@@ -388,17 +404,8 @@ int w4a4_gemm_s32(const int8_t* Xq, const int8_t* Wq, int32_t* acc, int64_t M, i
 int w4a4_linear_fused(const uint16_t* x, int64_t ldx, const int8_t* Wq, const float* sw, const uint16_t* bias,
                       uint16_t* y, int64_t ldy, int64_t M, int64_t N, int64_t K, int g, int act, void* workspace,
                       size_t workspace_bytes, void* stream) {
-  if (Wq == nullptr || sw == nullptr) return W4A4_ERR_NULL;
-  // an empty batch (M == 0) may pass NULL for its zero-size tensors
-  if (M != 0 && (x == nullptr || y == nullptr)) return W4A4_ERR_NULL;
-  int st = check_quant_shape(K, g);
+  int st = validate_fused(x, ldx, Wq, sw, bias, y, ldy, M, N, K, g, act);
   if (st != W4A4_OK) return st;
-  if (act != 0 && act != 1) return W4A4_ERR_ARG;
-  if ((st = check_gemm_shape(M, N, K)) != W4A4_OK) return st;
-  if (ldx < K || ldy < N) return W4A4_ERR_SHAPE;
-  if (ldx % 8 != 0 || !aligned(x, 16)) return W4A4_ERR_ALIGN;
-  if (ldy % 8 != 0 || !aligned(y, 16) || !aligned(Wq, 16) || !aligned(sw, 16)) return W4A4_ERR_ALIGN;
-  if (bias != nullptr && !aligned(bias, 16)) return W4A4_ERR_ALIGN;
   if (M == 0) {
     DeviceInfo* dev = nullptr;
     return current_device(&dev);

@@ -511,55 +511,3 @@ cudaError_t smallm_launch_tm(const CUtensorMap& tmW, const CUtensorMap& tmX, con
 int smallm_rows_padded(int64_t M) { return M <= 16 ? 16 : (M <= 32 ? 32 : 64); }
 
 }  // namespace w4a4
-
-// ---------------------------------------------------------------------------
-// Small-M linear that allocates nothing (w4a4_linear_noalloc in w4a4.h): the
-// small-M kernel reduces its K slices on chip and the tiny-M kernel keeps its
-// operands in one CTA, so neither needs scratch memory; this entry takes no
-// workspace argument.
-// ---------------------------------------------------------------------------
-#include "w4a4.h"
-
-extern "C" int w4a4_linear_noalloc(const int8_t* Xq, const float* sx, const int8_t* Wq, const float* sw,
-                                   const uint16_t* bias, uint16_t* y, int64_t M, int64_t N, int64_t K, int64_t ldy,
-                                   void* stream) {
-  using namespace w4a4;
-  int st = validate_linear(Xq, sx, Wq, sw, bias, y, M, N, K, ldy, 0);
-  if (st != W4A4_OK) return st;
-  if (M < 1 || M > kSmallMMax) return W4A4_ERR_SHAPE;
-  DeviceInfo* dev = nullptr;
-  if ((st = current_device(&dev)) != W4A4_OK) return st;
-  if (gemv_preferred(M, K)) {
-    // a few rows: the CUDA-core weight-streaming kernel, which needs no scratch either
-    GemvArgs g{};
-    g.xq = Xq;
-    g.sx = sx;
-    g.wq = Wq;
-    g.sw = sw;
-    g.bias = bias;
-    g.out = y;
-    g.M = M;
-    g.N = N;
-    g.K = K;
-    g.ldo = ldy;
-    g.out_s32 = 0;
-    return gemv_launch(g, dev->num_sms, static_cast<cudaStream_t>(stream)) == cudaSuccess ? W4A4_OK : W4A4_ERR_CUDA;
-  }
-  CUtensorMap tmW, tmX;
-  if ((st = packed_map(&tmW, Wq, N, K, WM, true)) != W4A4_OK) return st;
-  if ((st = packed_map(&tmX, Xq, M, K, smallm_rows_padded(M))) != W4A4_OK) return st;
-  SmallMArgs a{};
-  a.xq = Xq;
-  a.wq = Wq;
-  a.M = M;
-  a.N = N;
-  a.K = K;
-  a.sx = sx;
-  a.sw = sw;
-  a.bias = bias;
-  a.out = y;
-  a.ldo = ldy;
-  a.out_s32 = 0;
-  a.status = dev->status;
-  return smallm_launch_tm(tmW, tmX, a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? W4A4_OK : W4A4_ERR_CUDA;
-}

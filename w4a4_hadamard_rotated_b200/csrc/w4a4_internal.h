@@ -26,6 +26,9 @@ int group_rows_map(CUtensorMap* map, const uint16_t* x, int64_t M, int64_t K, in
 // Argument checks of w4a4_linear (out_s32 = 0) / w4a4_gemm_s32 (out_s32 = 1).
 int validate_linear(const int8_t* Xq, const float* sx, const int8_t* Wq, const float* sw, const uint16_t* bias,
                     const void* y, int64_t M, int64_t N, int64_t K, int64_t ldy, int out_s32);
+// Argument checks of w4a4_linear_fused (no CUDA call).
+int validate_fused(const uint16_t* x, int64_t ldx, const int8_t* Wq, const float* sw, const uint16_t* bias,
+                   const uint16_t* y, int64_t ldy, int64_t M, int64_t N, int64_t K, int g, int act);
 
 // ---- activation / weight rotate + quantise + pack (quant.cu)
 cudaError_t rotate_quant_bf16(const uint16_t* x, int64_t M, int K, int64_t ldx, int g, int act, int8_t* out,
