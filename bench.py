@@ -29,13 +29,21 @@ PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 INT8_OVER_BF16 = 2.0      # nominal dense int8 : bf16 tensor throughput on B200 (4.5 : 2.25 PFLOP/s)
 N_SETS = 5
-# DRAM bytes (read + write) per launch from ncu captures of the current
-# kernels, keyed by (kernel, workload); a kernel that changed since its
-# capture has no entry (traffic reported as null).  Figures: profiles/.
+REPEATS = 100             # timed regions per measured layer (each exactly --steps steps)
+# DRAM bytes per launch (dram__bytes_read.sum, dram__bytes_write.sum) of the
+# dominant kernel from one ncu capture of the current build, keyed by (kernel,
+# workload).  A kernel changed since its capture has no entry, and its
+# traffic is reported as null.  Outputs that still sit in L2 (126 MB) when a
+# kernel ends are written back during later kernels, so a capture's DRAM
+# writes miss them: such entries say so in "note".
 MEASURED_TRAFFIC = {
-    ("gemm_tc", "square"): 11.88e6 + 0.03e6,                 # profiles/gemm_tc_square_4608x3072x3072.md
-    ("smallm", "smallm_16_12288_3072"): 18.98e6 + 0.0,      # profiles/smallm_16x3072x12288.md
-    ("gemv", "smallm_1_12288_3072"): 18.95e6 + 0.0,         # profiles/gemv_1x3072x12288.md
+    ("gemm_tc", "square"): {
+        "read": 11_889_152, "write": 2_560,
+        "note": ("dram read+write of gemm_tc_kernel<0> per launch (ncu, square layer, 2 launches); the reads "
+                 "equal the algorithmic packed operands (Xq 7.08 MB + Wq 4.72 MB + scales); the 28.3 MB bf16 "
+                 "output is still in L2 when the kernel ends and reaches DRAM during later kernels, so it is "
+                 "not in this figure"),
+    },
 }
 
 
@@ -296,11 +304,35 @@ def time_graph(loop):
     return start.elapsed_time(end) / 1e3    # seconds
 
 
-def run_impl(args, cfg, world, rank, local):
-    import w4a4_hadamard_rotated_b200 as w4
-    w4.load_library()
+def time_regions(loop, repeats, world):
+    """`repeats` timed regions, each one replay of `loop` (exactly its steps),
+    bracketed by a barrier and a device synchronisation on both sides and
+    timed with CUDA events on the replay stream; each region's time is the
+    maximum over ranks.  Returns the list of region times in seconds."""
+    out = []
+    for _ in range(repeats):
+        torch.cuda.synchronize()
+        barrier(world)
+        dt = time_graph(loop)
+        torch.cuda.synchronize()
+        barrier(world)
+        out.append(max_over_ranks(dt, world))
+    return out
+
+
+def layer_roofline_s(cfg, peaks):
+    """The slower of 2MNK at the int8 tensor peak and the layer's algorithmic
+    bytes at the HBM peak."""
+    int8_peak = peaks.get("bf16_tflops", FALLBACK["bf16_tflops"]) * INT8_OVER_BF16
+    hbm = peaks.get("hbm_gbs", FALLBACK["hbm_gbs"])
+    return max(cfg.ops() / (int8_peak * 1e12), cfg.bytes() / (hbm * 1e9))
+
+
+def measure_layer(w4, cfg, args, world, repeats, sampler=None):
+    """One layer workload: its fused call timed over `repeats` regions of
+    exactly args.steps steps (CUDA-graph replays, rotating L2-cold operand
+    sets), and its two kernels alone (200-launch graphs, median of 5)."""
     device = torch.device("cuda", torch.cuda.current_device())
-    stream = torch.cuda.current_stream(device)
     sets = make_sets(cfg, w4, device)
     g = cfg.g
 
@@ -308,35 +340,17 @@ def run_impl(args, cfg, world, rank, local):
         s = sets[i % len(sets)]
         w4.linear_fused(s["x"], s["Wq"], s["sw"], s["b"], g, cfg.act, out=s["y"])
 
-    # ---- the timed region: exactly `steps` fused layer calls, replayed from
-    # CUDA graphs (the eager loop's time, host launch work included, is
-    # reported beside it)
     for i in range(args.warmup):
         fused(i)
     torch.cuda.synchronize()
     loop = GraphLoop(fused, args.steps)
     loop.run()   # one untimed replay
-    sampler = ClockSampler(device.index) if rank == 0 else None
     if sampler:
         sampler.start()
-    torch.cuda.synchronize()
-    barrier(world)
-    dt = time_graph(loop)
-    torch.cuda.synchronize()
-    barrier(world)
+    regions = time_regions(loop, repeats, world)
     clocks = sampler.stop() if sampler else None
-    dt_max = max_over_ranks(dt, world)
     del loop
-    dt_eager = max_over_ranks(time_loop(fused, args.steps, stream), world)
-    ops = float(cfg.ops())
-    value = world * ops * args.steps / dt_max / 1e12
-    ms_per_step = dt_max / args.steps * 1e3
-
-    # ---- per-kernel launch durations (the kernels and launch shapes the fused
-    # call runs, on the launching stream) for the roofline of the dominant kernel
-    path = w4.linear_kernel(cfg.M, cfg.N, cfg.K)   # the GEMM kernel linear() runs here
-    small = path != 0
-    gemm_name = {0: "gemm_tc", 1: "smallm", 3: "gemv"}[path]
+    dt_eager = max_over_ranks(time_loop(fused, args.steps, torch.cuda.current_stream(device)), world)
 
     def quant(i):
         s = sets[i % len(sets)]
@@ -346,15 +360,62 @@ def run_impl(args, cfg, world, rank, local):
         s = sets[i % len(sets)]
         w4.linear(s["Xq"], s["sx"], s["Wq"], s["sw"], s["b"], out=s["y"])
 
-
     reps = 200
     for i in range(3):
         quant(i)
         gemm(i)
-    t_quant = time_graph(GraphLoop(quant, reps)) / reps
+    ql = GraphLoop(quant, reps)
+    t_quant = statistics.median(time_graph(ql) for _ in range(5)) / reps
+    del ql
     for i in range(len(sets)):
         quant(i)
-    t_gemm = time_graph(GraphLoop(gemm, reps)) / reps
+    gl = GraphLoop(gemm, reps)
+    t_gemm = statistics.median(time_graph(gl) for _ in range(5)) / reps
+    del gl
+    per_step = [r / args.steps for r in regions]
+    return {"sets": sets, "per_step": per_step, "t_med": statistics.median(per_step), "t_min": min(per_step),
+            "t_eager": dt_eager / args.steps, "t_quant": t_quant, "t_gemm": t_gemm, "clocks": clocks}
+
+
+def layer_summary(w4, cfg, m, peaks):
+    """The per-layer keys of the JSON line."""
+    roof = layer_roofline_s(cfg, peaks)
+    path = w4.linear_kernel(cfg.M, cfg.N, cfg.K)
+    gemm_name = {0: "gemm_tc", 1: "smallm", 3: "gemv"}[path]
+    qpath = w4.quantize_activation_kernel(cfg.M, cfg.K, cfg.g, cfg.act)
+    return {
+        "workload": cfg.name,
+        "us_per_layer": m["t_med"] * 1e6, "us_per_layer_min": m["t_min"] * 1e6,
+        "us_per_layer_eager_launches": m["t_eager"] * 1e6,
+        "tops": cfg.ops() / m["t_med"] / 1e12,
+        "layer_roofline_us": roof * 1e6, "roofline_fraction_of_layer": roof / m["t_med"],
+        "kernels_us": {("rotate_quant_tc" if qpath == 2 else "rotate_quant_pack"): m["t_quant"] * 1e6,
+                       gemm_name: m["t_gemm"] * 1e6},
+        "timed_regions": len(m["per_step"]),
+    }
+
+
+def run_impl(args, cfg, world, rank, local):
+    import w4a4_hadamard_rotated_b200 as w4
+    w4.load_library()
+    device = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream(device)
+    peaks, kind = load_peaks()
+    g = cfg.g
+    repeats = max(1, args.repeats)
+
+    # ---- the timed region: `repeats` regions of exactly `steps` fused layer
+    # calls each, replayed from CUDA graphs; the value is the median region
+    sampler = ClockSampler(device.index) if rank == 0 else None
+    m = measure_layer(w4, cfg, args, world, repeats, sampler)
+    sets = m["sets"]
+    ops = float(cfg.ops())
+    value = world * ops / m["t_med"] / 1e12
+    ms_per_step = m["t_med"] * 1e3
+    t_quant, t_gemm = m["t_quant"], m["t_gemm"]
+    path = w4.linear_kernel(cfg.M, cfg.N, cfg.K)   # the GEMM kernel linear() runs here
+    small = path != 0
+    gemm_name = {0: "gemm_tc", 1: "smallm", 3: "gemv"}[path]
 
     # ---- end to end through the public API with host buffers: every step
     # copies its own x from pinned host memory, runs the fused layer and
@@ -404,6 +465,18 @@ def run_impl(args, cfg, world, rank, local):
     t_e2e = max_over_ranks(start.elapsed_time(end) / 1e3 / e2e_steps, world)
     e2e_value = world * ops / t_e2e / 1e12
     x_host, y_host = x_host[0], y_host[0]
+    del sets, m["sets"], s0, x_dev, y_dev
+
+    # ---- the other M = 4608 layers of the workload family, timed the same
+    # way (the default run covers every shape the 60% target applies to)
+    extra = {}
+    if args.workload == "square" and not args.no_extra_layers:
+        for name, c in (("mlp_up", workloads.MLP_UP), ("mlp_down", workloads.MLP_DOWN)):
+            mm = measure_layer(w4, c, args, world, repeats, ClockSampler(device.index) if rank == 0 else None)
+            extra[name] = layer_summary(w4, c, mm, peaks)
+            extra[name]["clocks"] = mm["clocks"]
+            del mm
+            torch.cuda.empty_cache()
 
     err = w4.last_device_error()
     if err != 0:
@@ -411,32 +484,36 @@ def run_impl(args, cfg, world, rank, local):
 
     if rank != 0:
         return
-    peaks, kind = load_peaks()
     burst = peaks.get("bf16_tflops", FALLBACK["bf16_tflops"])
     int8_peak = burst * INT8_OVER_BF16
     gemm_tops = ops / t_gemm / 1e12
     hbm = peaks.get("hbm_gbs", FALLBACK["hbm_gbs"])
     quant_bytes = 2 * cfg.M * cfg.K + cfg.M * cfg.K // 2 + 4 * cfg.M
-    roof_time = max(ops / (int8_peak * 1e12), cfg.bytes() / (hbm * 1e9))
+    roof_time = layer_roofline_s(cfg, peaks)
+    traffic = MEASURED_TRAFFIC.get((gemm_name, args.workload))
     if small:
         # weight streaming: the packed weight dominates the bytes
         k3_bytes = cfg.N * cfg.K // 2 + cfg.M * cfg.K // 2 + 4 * (cfg.M + cfg.N) + 2 * cfg.M * cfg.N
         roof = {"bound": "hbm", "achieved": k3_bytes / t_gemm / 1e9, "peak": hbm, "unit": "GB/s",
-                "frac": k3_bytes / t_gemm / 1e9 / hbm, "traffic": MEASURED_TRAFFIC.get((gemm_name, args.workload)),
+                "frac": k3_bytes / t_gemm / 1e9 / hbm,
                 "kernel": ("smallm_kernel (split-K weight streaming on the tensor cores)" if path == 1 else
                            "gemv_kernel (weight streaming on the CUDA cores)"),
                 "peak_note": f"{kind} HBM copy"}
     else:
         roof = {"bound": "tensor", "achieved": gemm_tops, "peak": int8_peak, "unit": "TOPS",
-                "frac": gemm_tops / int8_peak, "traffic": MEASURED_TRAFFIC.get(("gemm_tc", args.workload)),
+                "frac": gemm_tops / int8_peak,
                 "kernel": "gemm_tc_kernel (tcgen05 kind::i8, packed operands widened in shared memory, CTA pairs)",
                 "peak_note": f"int8 = 2 x {kind} bf16 burst {burst} TFLOP/s (nominal int8:bf16 ratio)"}
+    roof["traffic"] = None if traffic is None else traffic["read"] + traffic["write"]
+    if traffic is not None:
+        roof["traffic_note"] = traffic["note"]
     cpu = None
     if world == 1 or rank == 0:
         rows = min(256, cfg.M)
         t_cpu = time_oracle(cfg, rows)
         cpu = {"value": 2.0 * rows * cfg.N * cfg.K / t_cpu / 1e12, "unit": "TOPS", "cores": cpu_cores_used(),
                "kind": "oracle", "sample": f"{rows} of {cfg.M} rows, one pass, weights prepared offline"}
+    head = layer_summary(w4, cfg, m, peaks)
     line = {
         "metric": "W4A4 linear TOPS (fused quant+GEMM) at M=4608",
         "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -444,23 +521,28 @@ def run_impl(args, cfg, world, rank, local):
         "dtype": "s4xs4->s32", "data": "synthetic",
         "config": {"workload": cfg.name, "M": cfg.M, "K": cfg.K, "N": cfg.N, "g": cfg.g, "bias": cfg.bias,
                    "gelu_input": bool(cfg.act),
-                   "l2": f"{len(sets)} rotating input/weight/output sets (> 2x L2)",
+                   "l2": f"{n_sets_for(cfg)} rotating input/weight/output sets (> 2x L2)",
                    "launch": "CUDA graphs of the fused calls, replayed",
+                   "timing": (f"median of {repeats} timed regions of exactly {args.steps} steps each "
+                              "(CUDA events on the replay stream; barrier and synchronize around each region; "
+                              "max over ranks)"),
                    "parallelism": f"replicas x{world}"},
-        "us_per_layer": ms_per_step * 1e3,
-        "us_per_layer_eager_launches": dt_eager / args.steps * 1e6,
-        "roofline_fraction_of_layer": roof_time / (ms_per_step / 1e3),
-        "layer_roofline_us": roof_time * 1e6,
-        "kernels_us": {"rotate_quant_pack": t_quant * 1e6, gemm_name: t_gemm * 1e6},
+        "us_per_layer": head["us_per_layer"],
+        "us_per_layer_min": head["us_per_layer_min"],
+        "us_per_layer_eager_launches": head["us_per_layer_eager_launches"],
+        "roofline_fraction_of_layer": head["roofline_fraction_of_layer"],
+        "layer_roofline_us": head["layer_roofline_us"],
+        "kernels_us": head["kernels_us"],
         "roofline": roof,
         "quant_kernel_roofline": {"bound": "hbm", "achieved": quant_bytes / t_quant / 1e9, "peak": hbm,
                                   "unit": "GB/s", "frac": quant_bytes / t_quant / 1e9 / hbm},
+        "layers": extra,
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": "TOPS", "h2d_bytes_per_step": int(x_host.numel() * 2),
                 "d2h_bytes_per_step": int(y_host.numel() * 2),
                 "pipelining": "uploads, the fused layer and downloads on three streams, two buffers each"},
-        "gpu_launches": 2 * args.steps,
-        "clocks": clocks,
+        "gpu_launches": 2 * args.steps * repeats,
+        "clocks": m["clocks"],
     }
     print(json.dumps(line), flush=True)
 
@@ -554,9 +636,13 @@ def run_stack(args, g, world, rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=4000)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--repeats", type=int, default=REPEATS,
+                    help="timed regions of exactly --steps steps each; the value is their median")
+    ap.add_argument("--no-extra-layers", action="store_true",
+                    help="time only the named workload (the default square run also times MLP up and down)")
     ap.add_argument("--workload", default="square",
                     help="square (default: 4608x3072->3072), mlp_up, mlp_down, smallm_M_N_K, or stack_gG "
                          "(the 60-linear block stack at M=32760, group size G in 64/128/256)")

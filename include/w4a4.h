@@ -99,6 +99,27 @@ int w4a4_quantize_activation(const uint16_t* x, int64_t M, int64_t K, int64_t ld
                              int act, int8_t* Xq, float* sx, void* stream);
 
 /*
+ * w4a4_quantize_activation with the kernel chosen by the caller, for tests
+ * and measurements (both kernels compute the same page's rotation,
+ * quantisation and packing; they differ only in the order of the fp32
+ * additions of the rotation).
+ *   path 0: the routing of w4a4_quantize_activation (see
+ *           w4a4_quantize_activation_kernel);
+ *   path 1: the register-butterfly kernel (every shape);
+ *   path 2: the tensor-core kernel, for act = 0, g in {64, 128} and
+ *           K / g <= 128 (W4A4_ERR_SHAPE otherwise).
+ * Any other path gives W4A4_ERR_ARG.  Other arguments as above.
+ */
+int w4a4_quantize_activation_path(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int g,
+                                  int act, int8_t* Xq, float* sx, int path, void* stream);
+
+/* The kernel w4a4_quantize_activation (and the fused entries) run for this
+ * shape, as a path number of w4a4_quantize_activation_path (1 or 2); 0 for
+ * an invalid shape.  Pure host function; it reads the environment switches
+ * above. */
+int w4a4_quantize_activation_kernel(int64_t M, int64_t K, int g, int act);
+
+/*
  * W4A4 linear on already-quantised operands: the s4 x s4 GEMM with int32
  * accumulation and the rank-one epilogue of the page's Description (the row
  * and column scales are applied once per output, after the K loop).
@@ -197,6 +218,19 @@ int w4a4_linear_fused_noalloc(const uint16_t* x, int64_t ldx, const int8_t* Wq, 
  * W4A4_ERR_TIMEOUT, or W4A4_ERR_CUDA if the synchronisation failed.
  */
 int w4a4_last_device_error(void* stream);
+
+/*
+ * Test hook for the bounded waits of the product kernels: every kernel
+ * launched after this call (in this process, on any device) gives up a wait
+ * that has not ended after `limit_ns` nanoseconds, records W4A4_ERR_TIMEOUT
+ * in the device status word, stops every role, drains its copies and MMAs,
+ * frees its tensor memory and exits; its outputs are then undefined.  A
+ * limit of a few nanoseconds makes most waits expire at once.  0 restores
+ * the default of 2 s; values above 2 s or below 0 give W4A4_ERR_ARG.  Not
+ * for production use: it is process-wide and not synchronised with launches
+ * on other host threads.
+ */
+int w4a4_debug_set_wait_limit(int64_t limit_ns);
 
 /*
  * Test hook for the bounded-wait machinery: launches one CTA whose only

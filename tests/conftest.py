@@ -7,11 +7,6 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-# The tensor-core rotation serves 8192-row batches and up by default; the
-# parity cases of 512 rows and more reach it with this threshold (read once,
-# when the library first quantises).
-os.environ.setdefault("W4A4_ROTATE_TC_MIN_ROWS", "512")
-
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a B200 (sm_100a) and the built CUDA library")

@@ -198,3 +198,33 @@ def test_fused_noalloc_rejects_bad_arguments_and_oversized_shapes(lib):
     assert call(M=5448) == 2
     assert call(M=4608, K=12288, ldx=12288) == 2
     assert call(M=32760, K=5120, ldx=5120, N=5120, ldy=5120) == 2
+
+
+def test_quantize_activation_path_rejects_bad_arguments(lib):
+    q = lib.w4a4_quantize_activation_path
+    assert q(FAKE, 4, 256, 256, 128, 0, FAKE, FAKE, 3, NULL) == 9            # unknown path
+    assert q(FAKE, 4, 256, 256, 128, 0, FAKE, FAKE, -1, NULL) == 9
+    assert q(FAKE, 4, 256, 256, 128, 1, FAKE, FAKE, 2, NULL) == 2            # tensor cores: no GELU
+    assert q(FAKE, 4, 512, 512, 256, 0, FAKE, FAKE, 2, NULL) == 2            # tensor cores: g <= 128
+    assert q(FAKE, 4, 16384, 16384, 64, 0, FAKE, FAKE, 2, NULL) == 2         # tensor cores: K / g <= 128
+    assert q(NULL, 4, 256, 256, 128, 0, FAKE, FAKE, 1, NULL) == 1            # the common checks still apply
+
+
+def test_quantize_activation_kernel_routing(lib):
+    """Which activation kernel the entries run (a pure host function): the
+    register butterflies below 8192 rows and wherever the tensor-core form
+    does not apply, the tensor cores from 8192 rows up."""
+    f = lib.w4a4_quantize_activation_kernel
+    assert f(4608, 3072, 128, 0) == 1      # the M = 4608 layers
+    assert f(4608, 12288, 128, 1) == 1
+    assert f(8192, 3072, 128, 0) == 2
+    assert f(32760, 5120, 128, 0) == 2     # the block stack
+    assert f(32760, 5120, 256, 0) == 1     # g = 256: butterflies only
+    assert f(32760, 13824, 128, 1) == 1    # GELU input: butterflies only
+    assert f(4608, 3000, 128, 0) == 0      # invalid shape
+
+
+def test_debug_wait_limit_rejects_bad_values(lib):
+    assert lib.w4a4_debug_set_wait_limit(-1) == 9
+    assert lib.w4a4_debug_set_wait_limit(3_000_000_000) == 9
+    assert lib.w4a4_debug_set_wait_limit(0) == 0       # the default (2 s)

@@ -27,32 +27,61 @@ def _packed_cuda(q):
 # K1: rotate + quantise + pack
 # --------------------------------------------------------------------------
 
-@pytest.mark.parametrize("M,K,g,act", [
+def _tc_applies(K, g, act):
+    """Shapes the tensor-core rotation (quantiser path 2) takes."""
+    return act == 0 and g in (64, 128) and K // g <= 128
+
+
+_QUANT_CASES = [
     (16, 256, 128, 0), (333, 3072, 128, 0), (333, 3072, 64, 0), (333, 3072, 256, 0),
     (67, 12288, 128, 0), (67, 12288, 256, 1), (130, 5120, 64, 1), (1, 128, 128, 0), (5, 13824, 128, 0),
-    # 512 rows and more without activation take the tensor-core rotation (the
-    # threshold the test session sets)
-    # (whole rows per 128-lane tile: 5 x 24, 1 x 96, 3 x 40, 1 x 108, 2 x 48 lanes)
+    # tensor-core tiles of whole rows per 128 lanes: 5 x 24, 1 x 96, 3 x 40, 1 x 108, 2 x 48 lanes
     (777, 3072, 128, 0), (520, 12288, 128, 0), (513, 5120, 128, 0), (1000, 13824, 128, 0), (600, 3072, 64, 0),
     (700, 256, 128, 0),
     # one group per row (up to 128 rows per tile) and 128 groups per row (one row per tile)
     (40000, 128, 128, 0), (512, 8192, 64, 0),
-])
-def test_quantize_activation_parity(cuda_lib, M, K, g, act):
+]
+
+
+@pytest.mark.parametrize("M,K,g,act,path", [c + (p,) for c in _QUANT_CASES for p in (1, 2)
+                                            if p == 1 or _tc_applies(c[1], c[2], c[3])])
+def test_quantize_activation_parity(cuda_lib, M, K, g, act, path):
+    """Both activation kernels -- 1: register butterflies, 2: tensor cores --
+    against the oracle, chosen per call."""
     x = workloads.make_activation(M, K, seed=M + K + g, outlier_frac=0.005, outlier_scale=30.0)
-    Xq, sx = cuda_lib.quantize_activation(x.cuda(), g, act)
+    Xq, sx = cuda_lib.quantize_activation(x.cuda(), g, act, path=path)
     ref = orc.quantize_activation(workloads.bf16_bits(x), g, act)
-    check_packed(Xq, sx, ref, f"x {M}x{K} g{g} act{act}")
+    check_packed(Xq, sx, ref, f"x {M}x{K} g{g} act{act} path{path}", g, path)
 
 
-@pytest.mark.parametrize("M", [70, 700])
-def test_quantize_activation_strided_rows(cuda_lib, M):
+@pytest.mark.parametrize("M,K,act,path", [(4608, 3072, 0, 1), (4608, 3072, 0, 2), (4608, 12288, 0, 1),
+                                          (4608, 12288, 0, 2), (4608, 12288, 1, 1)])
+def test_quantize_activation_full_size(cuda_lib, M, K, act, path):
+    """Every row of the M = 4608 layers' activations (the square / MLP-up
+    input, and the MLP-down input with GELU) against the oracle, through the
+    kernel the layers run (path 1: the routing picks it at 4608 rows) and
+    through the tensor-core one.  At 4608 x 12288 each CTA of the register
+    kernel walks about eleven one-row tiles, so its shared-memory ring and
+    its row-amax slots wrap several times."""
+    g = 128
+    if path == 1:
+        assert cuda_lib.quantize_activation_kernel(M, K, g, act) == 1   # what the fused layer runs here
+    x = workloads.make_activation(M, K, seed=K + act, outlier_frac=0.005, outlier_scale=30.0)
+    if act == 1:
+        x = (x.float() * 3.0).to(torch.bfloat16)   # spread the GELU input over both tails
+    Xq, sx = cuda_lib.quantize_activation(x.cuda(), g, act, path=path)
+    ref = orc.quantize_activation(workloads.bf16_bits(x), g, act)
+    check_packed(Xq, sx, ref, f"x {M}x{K} act{act} path{path}", g, path)
+
+
+@pytest.mark.parametrize("M,path", [(70, 1), (700, 1), (70, 2), (700, 2)])
+def test_quantize_activation_strided_rows(cuda_lib, M, path):
     K, g = 1024, 128
     wide = workloads.make_activation(M, K + 64, seed=3, outlier_frac=0.01, outlier_scale=20.0).cuda()
     x = wide[:, :K]
-    Xq, sx = cuda_lib.quantize_activation(x, g)
+    Xq, sx = cuda_lib.quantize_activation(x, g, path=path)
     ref = orc.quantize_activation(workloads.bf16_bits(wide.cpu()[:, :K].contiguous()), g)
-    check_packed(Xq, sx, ref, "strided x")
+    check_packed(Xq, sx, ref, "strided x", g, path)
 
 
 @pytest.mark.parametrize("N,K,g", [(392, 512, 128), (128, 256, 64), (200, 3072, 256), (64, 12288, 128)])
@@ -60,17 +89,18 @@ def test_quantize_weight_parity(cuda_lib, N, K, g):
     W = workloads.make_weight(N, K, seed=N + K)
     Wq, sw = cuda_lib.quantize_weight(W.cuda(), g)
     ref = orc.quantize_weight(W.numpy(), g)
-    check_packed(Wq, sw, ref, f"W {N}x{K} g{g}")
+    check_packed(Wq, sw, ref, f"W {N}x{K} g{g}", g)
 
 
-def test_quantize_zero_rows(cuda_lib):
+@pytest.mark.parametrize("path", [1, 2])
+def test_quantize_zero_rows(cuda_lib, path):
     x = workloads.make_activation(40, 512, seed=9)
     x[[0, 7, 39]] = 0
-    Xq, sx = cuda_lib.quantize_activation(x.cuda(), 128)
+    Xq, sx = cuda_lib.quantize_activation(x.cuda(), 128, path=path)
     sx = sx.cpu()
     assert sx[0] == 0 and sx[7] == 0 and sx[39] == 0
     assert torch.all(Xq.cpu()[[0, 7, 39]] == 0)
-    check_packed(Xq, sx, orc.quantize_activation(workloads.bf16_bits(x), 128), "zero rows")
+    check_packed(Xq, sx, orc.quantize_activation(workloads.bf16_bits(x), 128), "zero rows", 128, path)
 
 
 def _one_hot_rows(t_bits, K=128):
@@ -205,7 +235,7 @@ def test_fused_tiny_m_matches_separate_calls(cuda_lib, M, K, g):
     assert torch.equal(scales.view(torch.int32), sx.view(torch.int32))
     assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
     ref = orc.quantize_activation(workloads.bf16_bits(x), g)
-    check_packed(codes, scales, ref, f"fused tiny {M}x{K} g{g}")
+    check_packed(codes, scales, ref, f"fused tiny {M}x{K} g{g}", g)
 
 
 def test_full_size_paths_agree(cuda_lib):
@@ -272,10 +302,11 @@ def _check_layer(cuda_lib, cfg, x, W, b, rows=None, y=None):
         y = cuda_lib.linear_fused(xc, Wq, sw, bc, cfg.g, cfg.act)
     Xq, sx = cuda_lib.quantize_activation(xc, cfg.g, cfg.act)
     wref, ref = _oracle_layer(cfg, x, W, b, rows)
-    check_packed(Wq, sw, wref, f"{cfg.name} weights")
+    check_packed(Wq, sw, wref, f"{cfg.name} weights", cfg.g)
     sel = slice(None) if rows is None else torch.as_tensor(rows)
     xa = orc.quantize_activation(workloads.bf16_bits(x if rows is None else x[rows]), cfg.g, cfg.act)
-    check_packed(Xq.cpu()[sel], sx.cpu()[sel], xa, f"{cfg.name} activations")
+    path = cuda_lib.quantize_activation_kernel(cfg.M, cfg.K, cfg.g, cfg.act)
+    check_packed(Xq.cpu()[sel], sx.cpu()[sel], xa, f"{cfg.name} activations", cfg.g, path)
     # the fused output equals the oracle epilogue on the GPU's own operands
     acc = orc.gemm_s32(Xq.cpu()[sel].numpy(), Wq.cpu().numpy())
     check_epilogue_exact(y.cpu()[sel], acc, sx.cpu()[sel].numpy(), sw.cpu().numpy(),
@@ -381,8 +412,53 @@ def test_bounded_wait_reports_timeout_and_context_survives(cuda_lib):
     _check_layer(cuda_lib, cfg, x, W, b)
 
 
-@pytest.mark.parametrize("n_rows", [300, 600])
-def test_quantize_exact_ties_follow_round_half_even(cuda_lib, n_rows):
+@pytest.mark.parametrize("kernel", ["quant_butterfly", "quant_tensor_core", "gemm_tc", "gemm_small_m",
+                                    "fused_square"])
+def test_product_kernel_waits_expire_and_context_survives(cuda_lib, kernel):
+    """With a wait limit of a few nanoseconds the product kernels' waits on
+    their copy rings, widened stages, accumulators and cluster peers expire
+    wherever they would have to wait: each kernel must record
+    W4A4_ERR_TIMEOUT, stop every role, let its copies and MMAs drain, free
+    its tensor memory and exit (its outputs are then undefined).  With the
+    default limit back, the same context runs the layer correctly."""
+    g = 128
+    big = workloads.make_activation(4608, 3072, seed=77, outlier_frac=0.005, outlier_scale=30.0).cuda()
+    Wbig = workloads.make_weight(3072, 3072, seed=78).cuda()
+    Wq, sw = cuda_lib.quantize_weight(Wbig, g)
+    Wk = workloads.make_weight(3072, 12288, seed=79).cuda()
+    Wqk, swk = cuda_lib.quantize_weight(Wk, g)
+    Xq, sx = cuda_lib.quantize_activation(big, g)
+    x16 = workloads.make_activation(16, 12288, seed=80).cuda()
+    Xq16, sx16 = cuda_lib.quantize_activation(x16, g)
+    torch.cuda.synchronize()
+    assert cuda_lib.last_device_error() == 0
+    runs = {
+        "quant_butterfly": lambda: cuda_lib.quantize_activation(big, g, path=1),
+        "quant_tensor_core": lambda: cuda_lib.quantize_activation(big, g, path=2),
+        "gemm_tc": lambda: cuda_lib.linear(Xq[:1000].contiguous(), sx[:1000].contiguous(), Wq, sw),
+        "gemm_small_m": lambda: cuda_lib.linear(Xq16, sx16, Wqk, swk),
+        "fused_square": lambda: cuda_lib.linear_fused(big, Wq, sw, None, g),
+    }
+    if kernel == "gemm_small_m":
+        assert cuda_lib.linear_kernel(16, 3072, 12288) == 1
+    try:
+        cuda_lib.debug_set_wait_limit(5)
+        runs[kernel]()
+        status = cuda_lib.last_device_error()
+    finally:
+        cuda_lib.debug_set_wait_limit(0)
+    assert status == 8                                  # W4A4_ERR_TIMEOUT, then cleared
+    assert cuda_lib.last_device_error() == 0
+    cfg = workloads.TINY
+    x, W, b = cfg.make()
+    _check_layer(cuda_lib, cfg, x, W, b)
+    y = cuda_lib.linear_fused(big, Wq, sw, None, g)     # and the full layer again
+    assert torch.equal(y.view(torch.int16), cuda_lib.linear(Xq, sx, Wq, sw).view(torch.int16))
+    assert cuda_lib.last_device_error() == 0
+
+
+@pytest.mark.parametrize("n_rows,path", [(300, 1), (600, 1), (300, 2), (600, 2)])
+def test_quantize_exact_ties_follow_round_half_even(cuda_lib, n_rows, path):
     """Rows built from the hand-derived tie fixture: every rotated value is an
     exact multiple of 1/2 or 1/4, so many codes sit exactly on a rounding
     boundary.  The kernel must decide all of them as round-half-even of the
@@ -404,7 +480,7 @@ def test_quantize_exact_ties_follow_round_half_even(cuda_lib, n_rows):
     xb = orc.f32_to_bf16_bits(X.astype(np.float32))
     assert np.array_equal(orc.bf16_bits_to_f32(xb).astype(np.float64), X)
     x = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).cuda()
-    Xq, sx = cuda_lib.quantize_activation(x, g)
+    Xq, sx = cuda_lib.quantize_activation(x, g, path=path)
     ref = orc.quantize_activation(xb, g)
     assert np.array_equal(Xq.cpu().numpy(), ref["packed"])
     assert np.array_equal(sx.cpu().numpy(), ref["scale"])

@@ -306,6 +306,44 @@ def test_gelu_saturates_at_both_ends():
     assert np.all(neg == 0.0) and np.all(np.signbit(neg))
 
 
+@pytest.mark.parametrize("t", [1.0, -1.0, 2.5])
+def test_activation_with_gelu_applies_gelu_before_the_rotation(t):
+    """A one-hot row (t in column 0, g = 64): GELU first turns t into
+    G = GELU(t), and the rotation then spreads G / 8 over the 64 outputs of
+    the first group (every entry of the first Hadamard column is +1, and
+    1/sqrt(64) = 1/8 is exact), so sx = fl(fl(G / 8) / 7) and the first
+    group's codes are all 7 * sign(G).  Rotating first would give
+    GELU(t / 8) instead: a different scale."""
+    G = np.float32(0.5 * t * (1.0 + math.erf(t / math.sqrt(2.0))))
+    want_s = np.float32(np.float32(G / np.float32(8.0)) / np.float32(7.0))
+    xb = np.zeros((1, 128), dtype=np.uint16)
+    xb[0, 0] = orc.f32_to_bf16_bits(np.array([t], dtype=np.float32))[0]
+    out = orc.quantize_activation(xb, 64, act=1)
+    assert out["scale"][0] == abs(want_s)
+    q = out["q"][0]
+    assert np.all(q[:64] == 7 * int(np.sign(G))) and np.all(q[64:] == 0)
+    # the other order is measurably different
+    other = np.float32(0.5 * (t / 8) * (1.0 + math.erf((t / 8) / math.sqrt(2.0))))
+    assert abs(np.float32(other / np.float32(7.0)) - abs(want_s)) > 1e-3 * abs(want_s)
+
+
+def test_activation_with_gelu_two_hot_row():
+    """Two inputs a, b in the columns 0 and 1 of a 64-group: after GELU the
+    rotation gives G(a) + G(b) on even outputs and G(a) - G(b) on odd ones
+    (Hadamard columns 0 and 1), divided by 8."""
+    a, b = 1.5, -0.75
+    Ga = 0.5 * a * (1.0 + math.erf(a / math.sqrt(2.0)))
+    Gb = 0.5 * b * (1.0 + math.erf(b / math.sqrt(2.0)))
+    xb = np.zeros((1, 64), dtype=np.uint16)
+    xb[0, :2] = orc.f32_to_bf16_bits(np.array([a, b], dtype=np.float32))
+    out = orc.quantize_activation(xb, 64, act=1)
+    Ga32, Gb32 = np.float64(np.float32(Ga)), np.float64(np.float32(Gb))
+    even, odd = (Ga32 + Gb32) / 8, (Ga32 - Gb32) / 8
+    assert np.allclose(out["r"][0, 0::2], even, rtol=1e-7, atol=0)
+    assert np.allclose(out["r"][0, 1::2], odd, rtol=1e-7, atol=0)
+    assert out["scale"][0] == np.float32(np.float32(max(abs(even), abs(odd))) / np.float32(7.0))
+
+
 # --------------------------------------------------------------------------
 # The whole layer
 # --------------------------------------------------------------------------

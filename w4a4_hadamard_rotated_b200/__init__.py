@@ -38,6 +38,8 @@ SIGNATURES = {
     "w4a4_version": (_I, []),
     "w4a4_quantize_weight": (_I, [_P, _I64, _I64, _I64, _I, _P, _P, _P]),
     "w4a4_quantize_activation": (_I, [_P, _I64, _I64, _I64, _I, _I, _P, _P, _P]),
+    "w4a4_quantize_activation_path": (_I, [_P, _I64, _I64, _I64, _I, _I, _P, _P, _I, _P]),
+    "w4a4_quantize_activation_kernel": (_I, [_I64, _I64, _I, _I]),
     "w4a4_linear": (_I, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P, _SZ, _P]),
     "w4a4_linear_fused": (_I, [_P, _I64, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I, _I, _P, _SZ, _P]),
     "w4a4_workspace_bytes": (_SZ, [_I64, _I64, _I64]),
@@ -48,6 +50,7 @@ SIGNATURES = {
 
     "w4a4_last_device_error": (_I, [_P]),
     "w4a4_debug_wait_timeout": (_I, [_I64, _P]),
+    "w4a4_debug_set_wait_limit": (_I, [_I64]),
 }
 
 _lib = None
@@ -97,6 +100,28 @@ def _need_cuda(t, dtype, name):
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
 
 
+def _need_out(t, dtype, shape, name, device):
+    """An output or operand tensor: on the same CUDA device, the given dtype
+    and shape, contiguous (the library takes raw pointers and fixed strides)."""
+    _need_cuda(t, dtype, name)
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _need_rows(t, dtype, rows, cols, name, device):
+    """A 2-D output with `rows` x `cols` and a contiguous inner dimension (its
+    row stride is passed to the library)."""
+    _need_cuda(t, dtype, name)
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if t.dim() != 2 or tuple(t.shape) != (rows, cols) or t.stride(1) != 1:
+        raise ValueError(f"{name} must be a [{rows}, {cols}] tensor with a contiguous inner dimension")
+
+
 def _bits(t):
     """View a bf16 tensor as its raw 16-bit patterns (no copy)."""
     return t.view(torch.int16)
@@ -138,8 +163,10 @@ def quantize_weight(W, g=128):
     return Wq, sw
 
 
-def quantize_activation(x, g=128, act=0, out=None):
-    """Rotate + quantise bf16 activations x [M, K] -> (Xq [M, K/2] int8, sx [M] fp32)."""
+def quantize_activation(x, g=128, act=0, out=None, path=None):
+    """Rotate + quantise bf16 activations x [M, K] -> (Xq [M, K/2] int8, sx [M] fp32).
+    path: None or 0 = the library's routing, 1 = the register-butterfly
+    kernel, 2 = the tensor-core kernel (w4a4_quantize_activation_path)."""
     lib = load_library()
     _need_cuda(x, torch.bfloat16, "x")
     if x.dim() != 2 or x.stride(1) != 1:
@@ -150,20 +177,48 @@ def quantize_activation(x, g=128, act=0, out=None):
         sx = torch.empty(M, dtype=torch.float32, device=x.device)
     else:
         Xq, sx = out
-    _check(lib.w4a4_quantize_activation(_ptr(x), M, K, x.stride(0), g, act, _ptr(Xq), _ptr(sx), _stream(x)),
-           "w4a4_quantize_activation")
+        _need_out(Xq, torch.int8, (M, K // 2), "Xq", x.device)
+        _need_out(sx, torch.float32, (M,), "sx", x.device)
+    if path is None:
+        st = lib.w4a4_quantize_activation(_ptr(x), M, K, x.stride(0), g, act, _ptr(Xq), _ptr(sx), _stream(x))
+    else:
+        st = lib.w4a4_quantize_activation_path(_ptr(x), M, K, x.stride(0), g, act, _ptr(Xq), _ptr(sx), path,
+                                               _stream(x))
+    _check(st, "w4a4_quantize_activation")
     return Xq, sx
+
+
+def quantize_activation_kernel(M, K, g=128, act=0):
+    """Which kernel quantize_activation() runs for this shape: 1 (register
+    butterflies) or 2 (tensor cores)."""
+    return int(load_library().w4a4_quantize_activation_kernel(M, K, g, act))
+
+
+def _check_packed_operands(Xq, Wq):
+    _need_cuda(Xq, torch.int8, "Xq")
+    _need_cuda(Wq, torch.int8, "Wq")
+    if Xq.dim() != 2 or Wq.dim() != 2 or Xq.shape[1] != Wq.shape[1]:
+        raise ValueError("Xq [M, K/2] and Wq [N, K/2] must be 2-D with the same packed width")
+    if not Xq.is_contiguous() or not Wq.is_contiguous():
+        raise ValueError("Xq and Wq must be contiguous (rows of K/2 bytes)")
+    if Wq.device != Xq.device:
+        raise ValueError("Xq and Wq must be on the same device")
 
 
 def linear(Xq, sx, Wq, sw, bias=None, out=None):
     """y [M, N] bf16 from quantised operands (int32 GEMM + rank-one epilogue)."""
     lib = load_library()
-    _need_cuda(Xq, torch.int8, "Xq")
-    _need_cuda(Wq, torch.int8, "Wq")
+    _check_packed_operands(Xq, Wq)
     M, Kh = Xq.shape
     N = Wq.shape[0]
     K = 2 * Kh
-    y = out if out is not None else torch.empty(M, N, dtype=torch.bfloat16, device=Xq.device)
+    dev = Xq.device
+    _need_out(sx, torch.float32, (M,), "sx", dev)
+    _need_out(sw, torch.float32, (N,), "sw", dev)
+    if bias is not None:
+        _need_out(bias, torch.bfloat16, (N,), "bias", dev)
+    y = out if out is not None else torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    _need_rows(y, torch.bfloat16, M, N, "out", dev)
     nbytes = lib.w4a4_workspace_bytes(M, N, K)
     ws = workspace(nbytes, Xq.device) if nbytes else None
     _check(lib.w4a4_linear(_ptr(Xq), _ptr(sx), _ptr(Wq), _ptr(sw), _ptr(bias), _ptr(y), M, N, K, y.stride(0),
@@ -171,13 +226,27 @@ def linear(Xq, sx, Wq, sw, bias=None, out=None):
     return y
 
 
+def _check_fused_operands(x, Wq, sw, bias):
+    _need_cuda(x, torch.bfloat16, "x")
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be a 2-D tensor with a contiguous inner dimension")
+    M, K = x.shape
+    _need_cuda(Wq, torch.int8, "Wq")
+    if Wq.dim() != 2 or Wq.shape[1] * 2 != K or not Wq.is_contiguous() or Wq.device != x.device:
+        raise ValueError("Wq must be a contiguous [N, K/2] int8 tensor on x's device")
+    N = Wq.shape[0]
+    _need_out(sw, torch.float32, (N,), "sw", x.device)
+    if bias is not None:
+        _need_out(bias, torch.bfloat16, (N,), "bias", x.device)
+    return M, K, N
+
+
 def linear_fused(x, Wq, sw, bias=None, g=128, act=0, out=None):
     """y [M, N] bf16 = the whole layer from bf16 activations x [M, K]."""
     lib = load_library()
-    _need_cuda(x, torch.bfloat16, "x")
-    M, K = x.shape
-    N = Wq.shape[0]
+    M, K, N = _check_fused_operands(x, Wq, sw, bias)
     y = out if out is not None else torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
+    _need_rows(y, torch.bfloat16, M, N, "out", x.device)
     nbytes = lib.w4a4_fused_workspace_bytes(M, N, K)
     ws = workspace(nbytes, x.device, "fused") if nbytes else None
     _check(lib.w4a4_linear_fused(_ptr(x), x.stride(0), _ptr(Wq), _ptr(sw), _ptr(bias), _ptr(y), y.stride(0),
@@ -190,12 +259,12 @@ def gemm_s32(Xq, Wq, path=0, out=None):
     kernel, 2: the warp-level mma.sync comparison kernel, 3: the tiny-M
     CUDA-core kernel, M <= 4)."""
     lib = load_library()
-    _need_cuda(Xq, torch.int8, "Xq")
-    _need_cuda(Wq, torch.int8, "Wq")
+    _check_packed_operands(Xq, Wq)
     M, Kh = Xq.shape
     N = Wq.shape[0]
     K = 2 * Kh
     acc = out if out is not None else torch.empty(M, N, dtype=torch.int32, device=Xq.device)
+    _need_rows(acc, torch.int32, M, N, "out", Xq.device)
     _check(lib.w4a4_gemm_s32(_ptr(Xq), _ptr(Wq), _ptr(acc), M, N, K, acc.stride(0), path, None, 0,
                              _stream(Xq)), "w4a4_gemm_s32")
     return acc
@@ -206,13 +275,18 @@ def linear_fused_noalloc(x, Wq, sw, bias=None, g=128, act=0, out=None):
     inside the library (see w4a4_linear_fused_noalloc in the header; calls
     that overlap on the GPU race on it)."""
     lib = load_library()
-    _need_cuda(x, torch.bfloat16, "x")
-    M, K = x.shape
-    N = Wq.shape[0]
+    M, K, N = _check_fused_operands(x, Wq, sw, bias)
     y = out if out is not None else torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
+    _need_rows(y, torch.bfloat16, M, N, "out", x.device)
     _check(lib.w4a4_linear_fused_noalloc(_ptr(x), x.stride(0), _ptr(Wq), _ptr(sw), _ptr(bias), _ptr(y), y.stride(0),
                                          M, N, K, g, act, _stream(x)), "w4a4_linear_fused_noalloc")
     return y
+
+
+def debug_set_wait_limit(limit_ns):
+    """Test hook: the bounded-wait limit of every kernel launched afterwards
+    (0 restores the default of 2 s); see w4a4_debug_set_wait_limit."""
+    _check(load_library().w4a4_debug_set_wait_limit(int(limit_ns)), "w4a4_debug_set_wait_limit")
 
 
 def last_device_error(device=None):

@@ -5,6 +5,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 #include <cstdlib>
 #include <mutex>
@@ -22,7 +23,10 @@ namespace {
 constexpr int kMaxDevices = 64;
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
+std::atomic<unsigned long long> g_wait_limit_ns{kWaitLimitNs};
 }  // namespace
+
+unsigned long long wait_limit_ns() { return g_wait_limit_ns.load(std::memory_order_relaxed); }
 
 // Resolve the current device; fills its SM count and the device address of
 // the status word on first use.
@@ -219,6 +223,8 @@ int run_linear(const int8_t* Xq, const float* sx, const int8_t* Wq, const float*
     a.ldo = ldo;
     a.out_s32 = out_s32;
     a.status = dev->status;
+    a.wait_ns = wait_limit_ns();
+    a.num_sms = dev->num_sms;
     a.early_w = early_w;
     return smallm_launch_tm(tmW, tmX, a, stream) == cudaSuccess ? W4A4_OK : W4A4_ERR_CUDA;
   }
@@ -241,6 +247,7 @@ int run_linear(const int8_t* Xq, const float* sx, const int8_t* Wq, const float*
   a.ldo = ldo;
   a.out_s32 = out_s32;
   a.status = dev->status;
+  a.wait_ns = wait_limit_ns();
   return gemm_tc_launch(tmA, tmB, tmY, a, dev->num_sms, stream) == cudaSuccess ? W4A4_OK : W4A4_ERR_CUDA;
 }
 
@@ -336,11 +343,24 @@ int w4a4_quantize_weight(const float* W, int64_t N, int64_t K, int64_t ldw, int 
 
 int w4a4_quantize_activation(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int g, int act, int8_t* Xq,
                              float* sx, void* stream) {
+  return w4a4_quantize_activation_path(x, M, K, ldx, g, act, Xq, sx, 0, stream);
+}
+
+int w4a4_quantize_activation_kernel(int64_t M, int64_t K, int g, int act) {
+  if (check_quant_shape(K, g) != W4A4_OK || (act != 0 && act != 1) || M < 0) return 0;
+  return rotate_quant_bf16_route(M, static_cast<int>(K), g, act);
+}
+
+int w4a4_quantize_activation_path(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int g, int act, int8_t* Xq,
+                                  float* sx, int path, void* stream) {
   // an empty batch (M == 0) may pass NULL for its zero-size tensors
   if (M != 0 && (x == nullptr || Xq == nullptr || sx == nullptr)) return W4A4_ERR_NULL;
   int st = check_quant_shape(K, g);
   if (st != W4A4_OK) return st;
   if (act != 0 && act != 1) return W4A4_ERR_ARG;
+  if (path < 0 || path > 2) return W4A4_ERR_ARG;
+  // the tensor-core rotation: bf16 rows without GELU, g in {64, 128}, K/g <= 128
+  if (path == 2 && (act != 0 || g == 256 || K / g > 128)) return W4A4_ERR_SHAPE;
   if (M < 0 || M > (int64_t(1) << 26)) return W4A4_ERR_SHAPE;
   if (ldx < K) return W4A4_ERR_SHAPE;
   if (ldx % 8 != 0 || !aligned(x, 16) || !aligned(Xq, 16) || !aligned(sx, 4)) return W4A4_ERR_ALIGN;
@@ -348,7 +368,7 @@ int w4a4_quantize_activation(const uint16_t* x, int64_t M, int64_t K, int64_t ld
   if ((st = current_device(&dev)) != W4A4_OK) return st;
   if (M == 0) return W4A4_OK;
   return rotate_quant_bf16(x, M, static_cast<int>(K), ldx, g, act, Xq, sx, dev->num_sms, dev->status,
-                           static_cast<cudaStream_t>(stream)) == cudaSuccess
+                           static_cast<cudaStream_t>(stream), path) == cudaSuccess
              ? W4A4_OK
              : W4A4_ERR_CUDA;
 }
@@ -438,6 +458,13 @@ int w4a4_last_device_error(void* stream) {
     if (cudaMemcpy(dev->status, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return W4A4_ERR_CUDA;
     return W4A4_ERR_TIMEOUT;
   }
+  return W4A4_OK;
+}
+
+int w4a4_debug_set_wait_limit(int64_t limit_ns) {
+  if (limit_ns < 0 || limit_ns > static_cast<int64_t>(kWaitLimitNs)) return W4A4_ERR_ARG;
+  g_wait_limit_ns.store(limit_ns == 0 ? kWaitLimitNs : static_cast<unsigned long long>(limit_ns),
+                        std::memory_order_relaxed);
   return W4A4_OK;
 }
 

@@ -340,7 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int t = cluster; t < tiles && ok; t += nclusters, ++lt) {
         const int ab = lt & 1;
-        if (!mbar_wait_cluster(&bars.acc_empty[ab], ((acc_ph >> ab) & 1) ^ 1, abort_flag, args.status)) {
+        if (!mbar_wait_cluster(&bars.acc_empty[ab], ((acc_ph >> ab) & 1) ^ 1, abort_flag, args.status, args.wait_ns)) {
           ok = false;
           break;
         }
@@ -348,7 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + ab * BN;
         for (int kb = 0; kb < num_kb; ++kb) {
-          if (!mbar_wait_cluster(&bars.wide_full[ws], wph, abort_flag, args.status)) {
+          if (!mbar_wait_cluster(&bars.wide_full[ws], wph, abort_flag, args.status, args.wait_ns)) {
             ok = false;
             break;
           }
@@ -376,7 +376,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int t = cluster; t < tiles; t += nclusters) {
         bool ok = true;
         for (int kb = 0; kb < num_kb; ++kb) {
-          if (!mbar_wait(&bars.wide_full[ws], wph, abort_flag, args.status)) { ok = false; break; }
+          if (!mbar_wait(&bars.wide_full[ws], wph, abort_flag, args.status, args.wait_ns)) { ok = false; break; }
           mbar_arrive_remote_smem(&bars.wide_full[ws], 0);
           if (++ws == SWD) { ws = 0; wph ^= 1; }
         }
@@ -392,7 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int t = cluster; t < tiles && ok; t += nclusters) {
         const int mb = t % num_m, nb = t / num_m;
         for (int kb = 0; kb < num_kb; ++kb) {
-          if (!mbar_wait(&bars.packed_empty[ps], ph ^ 1, abort_flag, args.status)) { ok = false; break; }
+          if (!mbar_wait(&bars.packed_empty[ps], ph ^ 1, abort_flag, args.status, args.wait_ns)) { ok = false; break; }
           mbar_arrive_expect_tx(&bars.packed_full[ps], kPStage);
           uint8_t* dst = smem + kOffPack + ps * kPStage;
           tma_load_2d(dst, &tmA, &bars.packed_full[ps], kb * BKP, mb * BM + static_cast<int>(rank) * HM);
@@ -401,8 +401,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (++ps == SP) { ps = 0; ph ^= 1; }
         }
       }
-      if (!ok) {
-        // let every copy this thread issued land before the CTA goes away
+      {
+        // Let every copy this thread issued land before the CTA goes away:
+        // after an abort some may never be consumed, and an abort raised by
+        // another role after this loop ended would otherwise go unnoticed here.
+        // In a normal run every phase waited for has completed already.
         for (int s2 = 0; s2 < SP && s2 < issued; ++s2) {
           const int64_t n_s = issued / SP + (s2 < issued % SP ? 1 : 0);
           (void)mbar_wait(&bars.packed_full[s2], static_cast<uint32_t>((n_s - 1) & 1), nullptr, nullptr, 100000000ull);
@@ -423,8 +426,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (++ws == SWD) { ws = 0; wph ^= 1; }
           continue;
         }
-        if (!warp_wait(&bars.packed_full[ps], ph, abort_flag, args.status) ||
-            !warp_wait_cluster(&bars.wide_empty[ws], wph ^ 1, abort_flag, args.status)) { ok = false; break; }
+        if (!warp_wait(&bars.packed_full[ps], ph, abort_flag, args.status, args.wait_ns) ||
+            !warp_wait_cluster(&bars.wide_empty[ws], wph ^ 1, abort_flag, args.status, args.wait_ns)) { ok = false; break; }
         widen_units(smem + kOffPack + ps * kPStage, smem + ws * kStage, wt);
         fence_async_shared();
         __syncwarp();
@@ -447,12 +450,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = cluster; t + nclusters < tiles; t += nclusters, ++lt) {
       const int ab = lt & 1;
       stage_scales(t, ab, et);
-      (void)warp_wait_cluster(&bars.acc_full[ab], (acc_ph >> ab) & 1, abort_flag, args.status);
+      (void)warp_wait_cluster(&bars.acc_full[ab], (acc_ph >> ab) & 1, abort_flag, args.status, args.wait_ns);
       acc_ph ^= 1u << ab;
       // staged scales visible to the four warps; every wait above is bounded, so
-      // all four always arrive here and then leave together on an abort
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      if (*abort_flag) break;
+      // all four always arrive here.  The barrier ORs their views of the abort
+      // flag, which another thread may raise at any moment, so all four leave
+      // together (and meet the same barriers below) or none does.
+      if (bar_sync_or(1, 128, *abort_flag != 0)) break;
       tc_fence_after();
       drain_chunks(t, ab, 0, BN / 32, epi_stage);
       tc_fence_before();
@@ -475,10 +479,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       stage_scales(t_last, ab, (warp & 3) * 32 + lane);
       // the last accumulator's phase: uses of buffer ab before it, mod 2
       (void)warp_wait_cluster(&bars.acc_full[ab], static_cast<uint32_t>((lt_last >> 1) & 1), abort_flag,
-                              args.status);
+                              args.status, args.wait_ns);
     }
-    asm volatile("bar.sync 2, 512;" ::: "memory");
-    if (*abort_flag == 0) {
+    // one verdict for all sixteen warps (nothing raises the flag after this
+    // barrier, but the OR makes the branch uniform by construction)
+    const bool aborted = bar_sync_or(2, 512, *abort_flag != 0);
+    if (!aborted) {
       tc_fence_after();
       const int part = warp >> 2;   // 0..3 within the lane quarter
       drain_chunks(t_last, ab, 2 * part, 2 * part + 2, smem + warp * 2 * kStageBox);

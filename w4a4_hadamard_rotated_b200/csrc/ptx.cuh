@@ -122,9 +122,10 @@ __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 __device__ __forceinline__ bool warp_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                                  unsigned int* status) {
+                                                  unsigned int* status,
+                                                  unsigned long long limit_ns = kWaitLimitNs) {
   bool ok = true;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait_cluster(bar, parity, abort, status);
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait_cluster(bar, parity, abort, status, limit_ns);
   __syncwarp();
   return __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
 }
@@ -133,11 +134,28 @@ __device__ __forceinline__ bool warp_wait_cluster(uint64_t* bar, uint32_t parity
 // shared-memory word), then __syncwarp orders the whole warp after lane 0's
 // acquire.  Returns the same verdict in every lane.  Call with all lanes.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          unsigned int* status) {
+                                          unsigned int* status, unsigned long long limit_ns = kWaitLimitNs) {
   bool ok = true;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort, status);
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort, status, limit_ns);
   __syncwarp();
   return __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
+}
+
+// Named barrier `id` over `nthreads` threads (a multiple of 32) that also
+// ORs `pred` across them: every participating thread gets the same answer,
+// so warps that branch on it (e.g. on an abort flag another thread may raise
+// at any time) all take the same branch and meet the same barriers later.
+__device__ __forceinline__ bool bar_sync_or(uint32_t id, uint32_t nthreads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.or.pred p, %2, %3, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"(pred ? 1u : 0u), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
 }
 
 // ------------------------------------------------- programmatic dependent launch

@@ -203,7 +203,7 @@ template <typename TIn, int G, int ACT>
 __global__ void __maxnreg__(96)
     rotate_quant_pack_kernel(const TIn* __restrict__ x, int64_t M, int K, int64_t ldx, int rows_per_tile,
                              int nstages, int8_t* __restrict__ out, float* __restrict__ scale,
-                             unsigned int* status) {
+                             unsigned int* status, unsigned long long wait_ns) {
   constexpr int C = InTraits<TIn>::kChunkElems;
   constexpr int NCH = kSlab / C;   // 16-byte chunks per slab
 
@@ -279,7 +279,7 @@ __global__ void __maxnreg__(96)
   for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
     const int st = it % nstages;
     const int64_t row = tile * P + p;
-    const bool ok = warp_wait(&full[st], static_cast<uint32_t>((it / nstages) & 1), &abort_flag, status);
+    const bool ok = warp_wait(&full[st], static_cast<uint32_t>((it / nstages) & 1), &abort_flag, status, wait_ns);
     const bool valid = active && row < M && ok;
 
     // Slot chunk j (j < NCH/2) fills the low halves of V[C*j .. C*j+C), slot
@@ -336,8 +336,11 @@ __global__ void __maxnreg__(96)
     const float amax = fmaxf(fmaxf(am[0], am[1]), fmaxf(am[2], am[3]));
     // max_k fl(|u_k| * norm) = fl(max_k |u_k| * norm): rounding is monotonic
     if (valid) atomicMax(&row_amax[it % 3][p], __float_as_uint(amax * norm));
-    __syncthreads();   // every thread has its slab: ring slot st is free again
-    if (abort_flag) break;
+    // Every thread has its slab: ring slot st is free again.  The barrier ORs
+    // the threads' views of the abort flag (a warp of this CTA may raise it in
+    // the next tile's wait while a slower one still reads it here), so all
+    // leave the loop at the same tile or none does.
+    if (__syncthreads_or(abort_flag != 0)) break;
     if (tid == 0) {
       const int64_t nt = tile + static_cast<int64_t>(nstages) * gridDim.x;
       if (nt < ntiles) {
@@ -527,7 +530,7 @@ static cudaError_t launch_rq(const TIn* x, int64_t M, int K, int64_t ldx, int8_t
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, kern, x, M, K, ldx, pl.P, pl.nst, out, scale, status);
+  e = cudaLaunchKernelEx(&cfg, kern, x, M, K, ldx, pl.P, pl.nst, out, scale, status, wait_limit_ns());
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -575,10 +578,19 @@ static int64_t rotate_tc_min_rows() {
   return v;
 }
 
+static bool tc_applies(int K, int g, int act) { return act == 0 && (g == 64 || g == 128) && K / g <= 128; }
+
+int rotate_quant_bf16_route(int64_t M, int K, int g, int act) {
+  return tc_applies(K, g, act) && M >= rotate_tc_min_rows() ? 2 : 1;
+}
+
 cudaError_t rotate_quant_bf16(const uint16_t* x, int64_t M, int K, int64_t ldx, int g, int act, int8_t* out,
-                              float* scale, int num_sms, unsigned int* status, cudaStream_t stream) {
-  if (act == 0 && (g == 64 || g == 128) && K / g <= 128 && M >= rotate_tc_min_rows())
+                              float* scale, int num_sms, unsigned int* status, cudaStream_t stream, int path) {
+  if (path == 0) path = rotate_quant_bf16_route(M, K, g, act);
+  if (path == 2) {
+    if (!tc_applies(K, g, act)) return cudaErrorNotSupported;
     return rotate_quant_bf16_tc(x, M, K, ldx, g, out, scale, num_sms, status, stream);
+  }
   if (act == 1) {
     const cudaError_t e = ensure_gelu_table();
     if (e != cudaSuccess) return e;

@@ -94,7 +94,8 @@ __device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
 template <int G>
 __global__ void __launch_bounds__(kThreadsTc, 2)
     rotate_quant_tc_kernel(const __grid_constant__ CUtensorMap tmX, int64_t M, int K, int rows_per_tile,
-                           int8_t* __restrict__ out, float* __restrict__ scale, unsigned int* status) {
+                           int8_t* __restrict__ out, float* __restrict__ scale, unsigned int* status,
+                           unsigned long long wait_ns) {
   using Lay = TcLayout<G>;
   extern __shared__ uint8_t smem_dyn[];
   __shared__ TcBars bars;
@@ -175,15 +176,18 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
       for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++issued) {
         const int s = issued % kStages;
         if (issued < kStages) continue;   // issued before the set-up
-        if (!mbar_wait(&bars.empty[s], ((issued / kStages) & 1) ^ 1, abort_flag, status)) break;
+        if (!mbar_wait(&bars.empty[s], ((issued / kStages) & 1) ^ 1, abort_flag, status, wait_ns)) break;
         mbar_arrive_expect_tx(&bars.full[s], Lay::kChunks * 128u * Gg * P);
 #pragma unroll
         for (int h = 0; h < Lay::kChunks; ++h)
           tma_load_3d(smem + Lay::kOffX + s * Lay::kStage + h * Lay::kChunkBytes, &tmX, &bars.full[s], h * 64, 0,
                       static_cast<int32_t>(t * P));
       }
-      if (*abort_flag) {
-        // let every copy this thread issued land before the CTA goes away
+      {
+        // Let every copy this thread issued land before the CTA goes away:
+        // after an abort some are never consumed, and an abort raised by
+        // another role after this loop ended would otherwise go unnoticed
+        // here.  In a normal run these phases have all completed already.
         for (int s = 0; s < kStages && s < issued; ++s) {
           const int n_s = issued / kStages + (s < issued % kStages ? 1 : 0);
           (void)mbar_wait(&bars.full[s], static_cast<uint32_t>((n_s - 1) & 1), nullptr, nullptr, 100000000ull);
@@ -198,8 +202,8 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
       for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++i) {
         const int s = i % kStages;
         const int b = i & 1;
-        if (!mbar_wait(&bars.acc_empty[b], ((i >> 1) & 1) ^ 1, abort_flag, status)) break;
-        if (!mbar_wait(&bars.full[s], (i / kStages) & 1, abort_flag, status)) break;
+        if (!mbar_wait(&bars.acc_empty[b], ((i >> 1) & 1) ^ 1, abort_flag, status, wait_ns)) break;
+        if (!mbar_wait(&bars.full[s], (i / kStages) & 1, abort_flag, status, wait_ns)) break;
         tc_fence_after();
         const uint32_t d = tmem_base + b * G;
 #pragma unroll
@@ -235,7 +239,7 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
       const int set = k % 3;
       // An expired wait makes every later one return at once; the group still
       // reaches its named barrier on every tile, so no warp is left waiting.
-      bool ok = *abort_flag == 0 && warp_wait(&bars.acc_full[b], (i >> 1) & 1, abort_flag, status);
+      bool ok = *abort_flag == 0 && warp_wait(&bars.acc_full[b], (i >> 1) & 1, abort_flag, status, wait_ns);
       ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;   // warp-uniform: the tensor-memory loads are collective
       tc_fence_after();
       const int64_t row = t * P + p;
@@ -360,7 +364,7 @@ cudaError_t launch_tc(const uint16_t* x, int64_t M, int K, int64_t ldx, int8_t* 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, rotate_quant_tc_kernel<G>, tm, M, K, P, out, scale, status);
+  e = cudaLaunchKernelEx(&cfg, rotate_quant_tc_kernel<G>, tm, M, K, P, out, scale, status, wait_limit_ns());
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

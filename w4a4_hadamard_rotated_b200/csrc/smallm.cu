@@ -226,7 +226,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       const int pre = args.early_w ? min(Lay::kSP, nkb) : 0;   // weight stages already in flight
       for (int kb = kb0; kb < kb1; ++kb) {
         if (kb - kb0 >= pre) {
-          if (!mbar_wait(&bars.empty[ps], ph ^ 1, abort_flag, args.status)) { ok = false; break; }
+          if (!mbar_wait(&bars.empty[ps], ph ^ 1, abort_flag, args.status, args.wait_ns)) { ok = false; break; }
           mbar_arrive_expect_tx(&bars.full[ps], Lay::kPackW + Lay::kPackX);
           tma_load_2d(smem + Lay::kOffPackW + ps * Lay::kPackW, &tmW, &bars.full[ps], kb * BKP, ntile * WM);
         }
@@ -234,7 +234,10 @@ __global__ void __launch_bounds__(kThreads, 2)
         ++issued;
         if (++ps == Lay::kSP) { ps = 0; ph ^= 1; }
       }
-      if (!ok) {
+      {
+        // every copy this thread issued lands before the CTA can exit (after an
+        // abort some are never consumed; in a normal run these phases have all
+        // completed already)
         for (int s = 0; s < Lay::kSP && s < issued; ++s) {
           const int n_s = issued / Lay::kSP + (s < issued % Lay::kSP ? 1 : 0);
           (void)mbar_wait(&bars.full[s], static_cast<uint32_t>((n_s - 1) & 1), nullptr, nullptr, 100000000ull);
@@ -247,7 +250,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       constexpr uint32_t idesc = idesc_i8(WM, NP);
       uint32_t ws = 0, wph = 0;
       for (int i = 0; i < nkb; ++i) {
-        if (!mbar_wait(&bars.wfull[ws], wph, abort_flag, args.status)) break;
+        if (!mbar_wait(&bars.wfull[ws], wph, abort_flag, args.status, args.wait_ns)) break;
         tc_fence_after();
         const uint64_t bd = sw128_kmajor_desc(smem_u32(smem + Lay::kOffWideX + ws * Lay::kWideX));
         const uint32_t a_tmem = tmem_base + kTmemA + ws * 32;
@@ -289,8 +292,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     for (int i = 0; i < nkb; ++i, ps = (ps + 1 == Lay::kSP ? 0 : ps + 1), ph ^= (ps == 0 ? 1u : 0u),
              ws = (ws + 1 == Lay::kST ? 0 : ws + 1), wph ^= (ws == 0 ? 1u : 0u)) {
       if (i % kGroups != grp) continue;
-      if (!warp_wait(&bars.full[ps], ph, abort_flag, args.status) ||
-          !warp_wait(&bars.wempty[ws], wph ^ 1, abort_flag, args.status)) { ok = false; break; }
+      if (!warp_wait(&bars.full[ps], ph, abort_flag, args.status, args.wait_ns) ||
+          !warp_wait(&bars.wempty[ws], wph ^ 1, abort_flag, args.status, args.wait_ns)) { ok = false; break; }
       {
         const uint8_t* src = smem + Lay::kOffPackW + ps * Lay::kPackW + r * BKP;
         const int swz = (r >> 1) & 3;
@@ -337,7 +340,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     // NP consecutive int32 values, its 16-byte chunk j stored at chunk
     // j ^ (r & kChunkMask), so the rows that go to one owner are contiguous.
     if (grp == 0) {
-      if (ok) (void)warp_wait(&bars.acc_full, 0, abort_flag, args.status);
+      if (ok) (void)warp_wait(&bars.acc_full, 0, abort_flag, args.status, args.wait_ns);
       if (*abort_flag == 0) {
         tc_fence_after();
         uint32_t acc[NP];
@@ -364,7 +367,10 @@ __global__ void __launch_bounds__(kThreads, 2)
   // (integer addition: exact in any order), applies the epilogue and writes
   // those outputs.  Nothing is read remotely, so no second barrier is needed:
   // an owner leaves only once every byte sent to it has landed, and a sender
-  // only once its copies have read its shared memory.
+  // only once its copies have read its shared memory.  That holds after an
+  // abort too: the expected byte count is armed before the barrier and every
+  // CTA pushes unconditionally after it, so the receive wait ignores the
+  // abort flag (and the debug wait limit) and always waits for the bytes.
   const int R = (WM + splits - 1) / splits;
   const int own_rows = min(WM - split * R, R);
   const uint32_t slot_bytes = static_cast<uint32_t>(R) * NP * 4;
@@ -384,7 +390,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     bulk_commit_group();
   }
   bool got = true;
-  if (splits > 1) got = warp_wait(&bars.recv_full, 0, abort_flag, args.status);
+  if (splits > 1) got = warp_wait(&bars.recv_full, 0, nullptr, args.status);
   if (got && *abort_flag == 0) {
     // item = (owned row, chunk of four activation rows); consecutive threads
     // take consecutive rows, so the stores of one activation row coalesce
@@ -448,11 +454,11 @@ void fill_cfg(cudaLaunchConfig_t* cfg, cudaLaunchAttribute* attr, int ctas, int 
 // Split plan: K slices per 128-row weight tile.  Two CTAs fit on an SM
 // (registers, shared memory and tensor memory each allow two), and clusters
 // pack into the GPCs with some loss, so the plan keeps the grid within 85% of
-// 2 x 148 CTAs -- every cluster is then resident at once (a second wave of a
+// 2 CTAs per SM (2 x 148 on a B200) -- every cluster is then resident at once (a second wave of a
 // few clusters would double the kernel's time) -- with at most kMaxSplits
 // slices and at least one k-block per slice.
-void smallm_plan(int64_t N, int64_t K, int* ntiles, int* kb_per, int* splits) {
-  constexpr int kMaxCtas = static_cast<int>(0.85 * 2 * 148);
+void smallm_plan(int64_t N, int64_t K, int num_sms, int* ntiles, int* kb_per, int* splits) {
+  const int kMaxCtas = static_cast<int>(0.85 * 2 * num_sms);
   const int nt = static_cast<int>((N + WM - 1) / WM);
   const int num_kb = static_cast<int>((K + BK - 1) / BK);
   int s = kMaxCtas / nt;
@@ -482,7 +488,7 @@ cudaError_t launch_cfg(const CUtensorMap& tmW, const CUtensorMap& tmX, const Sma
     attrs_set[dev] = true;
   }
   int nt, per, splits;
-  smallm_plan(a.N, a.K, &nt, &per, &splits);
+  smallm_plan(a.N, a.K, a.num_sms, &nt, &per, &splits);
   cudaLaunchConfig_t cfg;
   cudaLaunchAttribute attr[2];
   fill_cfg<NP, OUT_S32>(&cfg, attr, nt * splits, splits, stream);

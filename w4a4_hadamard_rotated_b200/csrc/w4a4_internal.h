@@ -17,6 +17,9 @@ struct DeviceInfo {
 };
 // The current device (must be sm_100); W4A4_OK or an error status.
 int current_device(DeviceInfo** out);
+// How long the kernels' bounded waits spin before they give up: kWaitLimitNs
+// (2 s), or the value set by w4a4_debug_set_wait_limit.
+unsigned long long wait_limit_ns();
 // TMA map over a packed int4 matrix [rows, K/2] bytes with box {64, box_rows}
 // (64-byte swizzle in shared memory when swizzle64).
 int packed_map(CUtensorMap* map, const int8_t* base, int64_t rows, int64_t K, int box_rows, bool swizzle64 = false);
@@ -31,8 +34,12 @@ int validate_fused(const uint16_t* x, int64_t ldx, const int8_t* Wq, const float
                    const uint16_t* y, int64_t ldy, int64_t M, int64_t N, int64_t K, int g, int act);
 
 // ---- activation / weight rotate + quantise + pack (quant.cu)
+// path: 0 = the routing of w4a4_quantize_activation, 1 = the register-butterfly
+// kernel, 2 = the tensor-core kernel (cudaErrorNotSupported where it does not apply).
 cudaError_t rotate_quant_bf16(const uint16_t* x, int64_t M, int K, int64_t ldx, int g, int act, int8_t* out,
-                              float* scale, int num_sms, unsigned int* status, cudaStream_t stream);
+                              float* scale, int num_sms, unsigned int* status, cudaStream_t stream, int path = 0);
+// Which kernel path 0 picks: 1 (register butterflies) or 2 (tensor cores).
+int rotate_quant_bf16_route(int64_t M, int K, int g, int act);
 cudaError_t rotate_quant_f32(const float* x, int64_t M, int K, int64_t ldx, int g, int8_t* out, float* scale,
                              int num_sms, unsigned int* status, cudaStream_t stream);
 // Tensor-core form of rotate_quant_bf16 for act = 0, g in {64, 128} and
@@ -55,6 +62,7 @@ struct GemmArgs {
   int64_t ldo;
   int out_s32;            // 1: raw int32 accumulators
   unsigned int* status;   // device status word (bounded-wait timeouts)
+  unsigned long long wait_ns;   // bounded-wait limit (wait_limit_ns())
 };
 // tmA: packed activations [M, K/2] bytes, tmB: packed weights [N, K/2] bytes,
 // both with box {64 bytes, kGemmBM/2 rows}; tmY: bf16 output [M, N] (row
@@ -82,6 +90,8 @@ struct SmallMArgs {
   int64_t ldo;
   int out_s32;
   unsigned int* status;   // device status word
+  unsigned long long wait_ns;   // bounded-wait limit (wait_limit_ns())
+  int num_sms;            // SMs of the device (the split plan keeps every cluster resident)
   // 1: the packed weights (and their scales) were complete before this
   // kernel started, so it may read them before its grid-dependency wait (set
   // by the fused entry, whose previous kernel is its own activation
