@@ -150,7 +150,7 @@ __device__ __forceinline__ void widen_units(const uint8_t* __restrict__ pstage, 
 #pragma unroll
   for (int i = 0; i < kUnitsPerThread; ++i) {
     const int u = wt + i * kWidenThreads;
-    if (u < kUnits) buf[i] = *reinterpret_cast<const uint4*>(pstage + u * 16);
+    if (u < kUnits) buf[i] = lds128(smem_u32(pstage) + u * 16);
   }
 #pragma unroll
   for (int i = 0; i < kUnitsPerThread; ++i) {
@@ -165,10 +165,10 @@ __device__ __forceinline__ void widen_units(const uint8_t* __restrict__ pstage, 
     widen_word16(buf[i].y, c0.z, c0.w);
     widen_word16(buf[i].z, c1.x, c1.y);
     widen_word16(buf[i].w, c1.z, c1.w);
-    uint8_t* rowp = stage + (isA ? 0 : kWideA) + (r >> 3) * 1024 + (r & 7) * 128;
+    const uint32_t rowp = smem_u32(stage) + (isA ? 0 : kWideA) + (r >> 3) * 1024 + (r & 7) * 128;
     const int sw = r & 7;
-    *reinterpret_cast<uint4*>(rowp + (((2 * part) ^ sw) << 4)) = c0;
-    *reinterpret_cast<uint4*>(rowp + (((2 * part + 1) ^ sw) << 4)) = c1;
+    sts128(rowp + (((2 * part) ^ sw) << 4), c0);
+    sts128(rowp + (((2 * part + 1) ^ sw) << 4), c1);
   }
 }
 
@@ -180,7 +180,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ Bars bars;
   __shared__ __align__(16) float epi_sw[2][BN];
   __shared__ __align__(16) float epi_bias[2][BN];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = align1024_shared(smem_dyn);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;

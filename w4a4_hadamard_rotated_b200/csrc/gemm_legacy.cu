@@ -62,7 +62,7 @@ __global__ void __launch_bounds__(kLThreads, 1)
   extern __shared__ uint8_t smem_dyn[];
   __shared__ uint64_t full[LS], empty[LS];
   __shared__ int abort_flag;
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = align1024_shared(smem_dyn);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int num_n = static_cast<int>((N + LT - 1) / LT);
   const int mb = blockIdx.x / num_n, nb = blockIdx.x % num_n;

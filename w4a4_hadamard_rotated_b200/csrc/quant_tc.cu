@@ -99,7 +99,7 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
   using Lay = TcLayout<G>;
   extern __shared__ uint8_t smem_dyn[];
   __shared__ TcBars bars;
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = align1024_shared(smem_dyn);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int P = rows_per_tile;
