@@ -547,6 +547,59 @@ def run_impl(args, cfg, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+def run_nsplit(args, cfg, world, rank):
+    """The layer split over the ranks along its output features (weight
+    rows), every rank computing its column block with the library's kernels
+    and an all-gather (NCCL) assembling y on every rank: strong scaling of
+    one layer.  Timed eagerly (the all-gather is a NCCL call per step) over
+    `repeats` regions of exactly `steps` steps; the value is the median."""
+    import w4a4_hadamard_rotated_b200 as w4
+    from w4a4_hadamard_rotated_b200 import nsplit
+    w4.load_library()
+    device = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream(device)
+    sets = make_sets(cfg, w4, device)
+    layers = [nsplit.NSplitLinear(s["Wq"], s["sw"], s["b"], cfg.g) for s in sets]
+
+    def step(i):
+        k = i % len(sets)
+        layers[k](sets[k]["x"], cfg.act, out=sets[k]["y"])
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(device.index) if rank == 0 else None
+    if sampler:
+        sampler.start()
+    regions = []
+    for _ in range(max(1, args.repeats)):
+        torch.cuda.synchronize()
+        barrier(world)
+        regions.append(max_over_ranks(time_loop(step, args.steps, stream), world))
+        torch.cuda.synchronize()
+        barrier(world)
+    clocks = sampler.stop() if sampler else None
+    err = w4.last_device_error()
+    if err != 0:
+        raise RuntimeError(f"device status {err} after the benchmark")
+    if rank != 0:
+        return
+    t = statistics.median(regions) / args.steps
+    peaks, kind = load_peaks()
+    line = {
+        "metric": "W4A4 linear TOPS (fused quant+GEMM) at M=4608, output features split over the GPUs",
+        "value": cfg.ops() / t / 1e12, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True, "scaling": "strong",
+        "vs_baseline": None, "dtype": "s4xs4->s32", "data": "synthetic",
+        "config": {"workload": cfg.name, "M": cfg.M, "K": cfg.K, "N": cfg.N, "g": cfg.g,
+                   "parallelism": f"N-split x{world} + all-gather of y",
+                   "timing": f"median of {len(regions)} eager regions of exactly {args.steps} steps"},
+        "us_per_layer": t * 1e6, "layer_roofline_us_one_gpu": layer_roofline_s(cfg, peaks) * 1e6,
+        "gpu_launches": 2 * args.steps * len(regions), "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def run_stack(args, g, world, rank):
     """The transformer-block linear stack at M = 32760 (10 blocks of q, k, v,
     out 5120x5120 and an MLP 5120->13824->5120): per block one quantised
@@ -641,6 +694,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--repeats", type=int, default=REPEATS,
                     help="timed regions of exactly --steps steps each; the value is their median")
+    ap.add_argument("--parallel", default="replicas", choices=["replicas", "nsplit"],
+                    help="replicas: every GPU runs the whole layer on its own batch (weak scaling, the default); "
+                         "nsplit: one layer's output features split over the GPUs with an all-gather (strong)")
     ap.add_argument("--no-extra-layers", action="store_true",
                     help="time only the named workload (the default square run also times MLP up and down)")
     ap.add_argument("--workload", default="square",
@@ -667,6 +723,8 @@ def main():
     try:
         if args.impl == "reference":
             run_reference(args, cfg, world, rank)
+        elif args.parallel == "nsplit":
+            run_nsplit(args, cfg, world, rank)
         else:
             run_impl(args, cfg, world, rank, local)
     finally:
