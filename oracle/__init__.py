@@ -15,6 +15,9 @@ Sources (web pages on the method; cited by page title and section):
     ConvRot with a configurable group size.
   * "ComfyUI-INT4-Fast Introduction" (runcomfy), section "How ComfyUI-INT4-Fast
     Works" -- what the rotation is for.
+  * "Comfy-INT4-HIPtest README", section "LoRA modes", and "ComfyUI-INT4-Fast"
+    (features list, "Dynamic LoRA Patching") -- the Dynamic LoRA delta, with
+    the down projection rotated into the layer's basis.
 Where these pages leave a constant open (the 1/sqrt(g) normalisation, the
 scale amax/7, round-half-to-even, the [-7, 7] clamp, the fp32 rank-one
 epilogue) the oracle follows the layer's written specification, and every
@@ -41,4 +44,6 @@ from .w4a4_oracle import (  # noqa: F401
     epilogue,
     linear,
     boundary_window,
+    lora_delta,
+    linear_lora,
 )

@@ -233,3 +233,46 @@ def linear(x_bits, wq_packed, sw, bias_bits, g, act=0):
     y32, ybits = epilogue(acc, xa["scale"], sw, bias_bits)
     return {"xq": xa["packed"], "sx": xa["scale"], "v": xa["v"],
             "acc": acc, "y32": y32, "y_bits": ybits}
+
+
+# ---------------------------------------------------------------------------
+# Dynamic LoRA.  Page "Comfy-INT4-HIPtest README", section "LoRA modes": the
+# Dynamic mode keeps the LoRA matrices separate and applies their deltas at
+# inference time.  Page "ComfyUI-INT4-Fast" (features list, "Dynamic LoRA
+# Patching"): the LoRA down projection is rotated with the same Hadamard
+# transform as the layer, so that it stays coherent with the rotated basis.
+# ---------------------------------------------------------------------------
+
+
+def lora_delta(x_bits, A, B, g, scale, act=0):
+    """The LoRA delta of one layer in the rotated basis, in float64:
+    t = x_rot A_rot^T (the rotated activation against the rotated down
+    projection A [r, K]), delta = scale * t B^T (B [N, r], the up
+    projection).  x_rot and A_rot are the rows rotated blockwise exactly as
+    the layer rotates them (u / sqrt(g), not rounded); the activation is the
+    layer's input, i.e. GELU(x) when act = 1.
+
+    Returns (t [M, r], delta [M, N]), both float64."""
+    xf = bf16_bits_to_f32(x_bits)
+    if act == 1:
+        xf = gelu_f32(xf)
+    elif act != 0:
+        raise ValueError("act must be 0 (none) or 1 (gelu)")
+    sg = np.sqrt(np.float64(g))
+    ux, _ = rotate_rows(xf.astype(np.float64), g)
+    ua, _ = rotate_rows(np.asarray(A, dtype=np.float64), g)
+    t = (ux / sg) @ (ua / sg).T
+    delta = np.float64(scale) * (t @ np.asarray(B, dtype=np.float64).T)
+    return t, delta
+
+
+def linear_lora(x_bits, wq_packed, sw, bias_bits, g, A, B, scale, act=0):
+    """The layer with a dynamic LoRA: the W4A4 layer's fp32 output (the
+    rank-one epilogue of `linear`) plus the fp32-rounded delta, then one
+    round-to-nearest-even to bf16."""
+    base = linear(x_bits, wq_packed, sw, bias_bits, g, act)
+    t, delta = lora_delta(x_bits, A, B, g, scale, act)
+    y32 = (base["y32"] + delta.astype(np.float32)).astype(np.float32)
+    out = dict(base)
+    out.update({"t": t, "delta": delta, "base_y32": base["y32"], "y32": y32, "y_bits": f32_to_bf16_bits(y32)})
+    return out

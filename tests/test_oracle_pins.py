@@ -374,3 +374,80 @@ def test_linear_zero_activation_gives_bias():
     bias = workloads.bf16_bits(workloads.make_bias(8, 0))
     out = orc.linear(xb, wq["packed"], wq["scale"], bias, 64)
     assert np.array_equal(out["y_bits"], np.broadcast_to(bias, (3, 8)))
+
+
+# --------------------------------------------------------------------------
+# Dynamic LoRA
+# --------------------------------------------------------------------------
+
+def _lora_case(M=5, K=256, N=24, r=8, g=64, seed=3):
+    gen = np.random.default_rng(seed)
+    x = workloads.make_activation(M, K, seed=seed, outlier_frac=0.02, outlier_scale=10.0)
+    A = gen.standard_normal((r, K)).astype(np.float32) * 0.05
+    B = gen.standard_normal((N, r)).astype(np.float32) * 0.05
+    return workloads.bf16_bits(x), A, B
+
+
+@pytest.mark.parametrize("g", [64, 128, 256])
+def test_lora_rotated_delta_equals_the_unrotated_one(g):
+    """(H/sqrt(g))^2 = I: the rotated activation against the rotated down
+    projection gives x A^T, so the rotated delta equals the plain LoRA delta
+    (float64, 1e-12).  Rotating A with another group size, or not at all,
+    breaks this."""
+    xb, A, B = _lora_case(K=512, g=g)
+    t, delta = orc.lora_delta(xb, A, B, g, 0.75)
+    x = orc.bf16_bits_to_f32(xb).astype(np.float64)
+    t_plain = x @ A.astype(np.float64).T
+    assert np.allclose(t, t_plain, rtol=1e-12, atol=1e-12 * np.abs(t_plain).max())
+    d_plain = 0.75 * t_plain @ B.astype(np.float64).T
+    assert np.allclose(delta, d_plain, rtol=1e-12, atol=1e-12 * np.abs(d_plain).max())
+    # a down projection rotated with the wrong group size is not coherent
+    _, ua = orc.rotate_rows(A.astype(np.float64), g // 2)
+    ux, _ = orc.rotate_rows(x, g)
+    wrong = (ux / np.sqrt(g)) @ (ua / np.sqrt(g // 2)).T
+    assert not np.allclose(wrong, t_plain, rtol=1e-3)
+
+
+def test_lora_delta_brute_force():
+    """Tiny case written out with explicit Hadamard sums in Python."""
+    xb, A, B = _lora_case(M=2, K=128, N=3, r=2, g=64, seed=9)
+    t, delta = orc.lora_delta(xb, A, B, 64, 2.0)
+    x = orc.bf16_bits_to_f32(xb).astype(np.float64)
+    H = scipy.linalg.hadamard(64)
+
+    def rot(v):
+        out = []
+        for b0 in range(0, len(v), 64):
+            for i in range(64):
+                out.append(sum(H[i][j] * float(v[b0 + j]) for j in range(64)) / 8.0)
+        return out
+
+    for m in range(2):
+        xr = rot(x[m])
+        for j in range(2):
+            ar = rot(A[j].astype(np.float64))
+            assert abs(t[m, j] - sum(a * b for a, b in zip(xr, ar))) <= 1e-12 * max(1.0, abs(t[m, j]))
+        for n in range(3):
+            want = 2.0 * sum(t[m, j] * float(B[n, j]) for j in range(2))
+            assert abs(delta[m, n] - want) <= 1e-12 * max(1.0, abs(want))
+
+
+def test_lora_zero_update_gives_the_base_layer():
+    xb, A, B = _lora_case()
+    w = workloads.make_weight(24, 256, 0).numpy()
+    wq = orc.quantize_weight(w, 64)
+    bias = workloads.bf16_bits(workloads.make_bias(24, 0))
+    base = orc.linear(xb, wq["packed"], wq["scale"], bias, 64)
+    for Bz, s in ((np.zeros_like(B), 1.0), (B, 0.0)):
+        out = orc.linear_lora(xb, wq["packed"], wq["scale"], bias, 64, A, Bz, s)
+        assert np.array_equal(out["y_bits"], base["y_bits"])
+    out = orc.linear_lora(xb, wq["packed"], wq["scale"], bias, 64, A, B, 1.0)
+    assert not np.array_equal(out["y_bits"], base["y_bits"])
+    assert np.array_equal(out["y32"], (base["y32"] + out["delta"].astype(np.float32)).astype(np.float32))
+
+
+def test_lora_with_gelu_input_uses_gelu_of_x():
+    xb, A, B = _lora_case()
+    t1, _ = orc.lora_delta(xb, A, B, 64, 1.0, act=1)
+    xg = orc.gelu_f32(orc.bf16_bits_to_f32(xb)).astype(np.float64)
+    assert np.allclose(t1, xg @ A.astype(np.float64).T, rtol=1e-12, atol=1e-12)
