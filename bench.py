@@ -377,6 +377,48 @@ def measure_layer(w4, cfg, args, world, repeats, sampler=None):
             "t_eager": dt_eager / args.steps, "t_quant": t_quant, "t_gemm": t_gemm, "clocks": clocks}
 
 
+def measure_lora(w4, cfg, args, world, repeats, peaks, r=64):
+    """The layer with a Dynamic LoRA update of rank r (synthetic bf16 A, B
+    ~ N(0, 0.02), scale 16 / r): the fused LoRA layer timed like the plain
+    layer, and the LoRA update alone (down projection + up projection added
+    to y) with its algorithmic bytes against the HBM peak."""
+    device = torch.device("cuda", torch.cuda.current_device())
+    sets = make_sets(cfg, w4, device)
+    gen = torch.Generator().manual_seed(1234)
+    loras = [((torch.randn(r, cfg.K, generator=gen) * 0.02).to(torch.bfloat16).to(device),
+              (torch.randn(cfg.N, r, generator=gen) * 0.02).to(torch.bfloat16).to(device)) for _ in sets]
+    scale = 16.0 / r
+
+    def fused(i):
+        k = i % len(sets)
+        s = sets[k]
+        w4.linear_fused_lora(s["x"], s["Wq"], s["sw"], s["b"], loras[k][0], loras[k][1], scale, cfg.g, out=s["y"])
+
+    def upd(i):
+        k = i % len(sets)
+        w4.lora_add(sets[k]["x"], loras[k][0], loras[k][1], scale, sets[k]["y"])
+
+    for i in range(args.warmup):
+        fused(i)
+    torch.cuda.synchronize()
+    loop = GraphLoop(fused, args.steps)
+    loop.run()
+    per_step = [t / args.steps for t in time_regions(loop, repeats, world)]
+    del loop
+    ul = GraphLoop(upd, 200)
+    t_upd = statistics.median(time_graph(ul) for _ in range(5)) / 200
+    del ul
+    hbm = peaks.get("hbm_gbs", FALLBACK["hbm_gbs"])
+    upd_bytes = (2 * cfg.M * cfg.K + 2 * r * cfg.K + 2 * cfg.M * 64) + (2 * cfg.M * 64 + 2 * cfg.N * r + 4 * cfg.M * cfg.N)
+    t_med = statistics.median(per_step)
+    return {"workload": f"{cfg.name} + dynamic LoRA r={r}", "rank": r, "us_per_layer": t_med * 1e6,
+            "us_per_layer_min": min(per_step) * 1e6, "timed_regions": len(per_step),
+            "lora_update_us": t_upd * 1e6,
+            "lora_update_roofline": {"bound": "hbm", "bytes": upd_bytes, "achieved": upd_bytes / t_upd / 1e9,
+                                     "peak": hbm, "unit": "GB/s", "frac": upd_bytes / t_upd / 1e9 / hbm,
+                                     "kernels": "lora_down_kernel (t = x A^T) + lora_up_kernel (y += scale t B^T)"}}
+
+
 def layer_summary(w4, cfg, m, peaks):
     """The per-layer keys of the JSON line."""
     roof = layer_roofline_s(cfg, peaks)
@@ -477,6 +519,10 @@ def run_impl(args, cfg, world, rank, local):
             extra[name]["clocks"] = mm["clocks"]
             del mm
             torch.cuda.empty_cache()
+
+    if args.workload == "square" and not args.no_extra_layers:
+        extra["square_dynamic_lora_r64"] = measure_lora(w4, cfg, args, world, repeats, peaks)
+        torch.cuda.empty_cache()
 
     err = w4.last_device_error()
     if err != 0:

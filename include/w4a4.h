@@ -213,6 +213,44 @@ int w4a4_linear_fused_noalloc(const uint16_t* x, int64_t ldx, const int8_t* Wq, 
                               int g, int act, void* stream);
 
 /*
+ * Dynamic LoRA (page "Comfy-INT4-HIPtest README", section "LoRA modes":
+ * Dynamic keeps the LoRA matrices separate and applies their deltas at
+ * inference time; page "ComfyUI-INT4-Fast", "Dynamic LoRA Patching": the
+ * down projection is rotated into the layer's Hadamard basis).  Adds
+ *     y[m, n] += scale * sum_j t[m, j] B[n, j],   t = x_rot A_rot^T = x A^T
+ * to an existing bf16 output: the rotation is orthogonal, so the rotated
+ * activation against the rotated down projection equals the plain product,
+ * which the kernels form from the bf16 activation and the unrotated A.
+ *   x [M, K] bf16 bits, row stride ldx >= K, ldx % 8 == 0 (the layer's input)
+ *   A [r, K] bf16 bits (the down projection, contiguous rows)
+ *   B [N, r] bf16 bits (the up projection, contiguous rows)
+ *   r in {16, 32, 48, 64};  scale finite (e.g. alpha / r)
+ *   y [M, N] bf16 bits, row stride ldy >= N, ldy % 8 == 0; updated in place:
+ *       y = bf16(fma(scale, delta, y)) with delta accumulated in fp32 from
+ *       bf16 t (t itself accumulated in fp32 from bf16 products)
+ *   M >= 0, N % 8 == 0, K % 8 == 0;  every pointer 16-byte aligned
+ *   workspace: at least w4a4_lora_workspace_bytes(M, K) bytes, 256-byte
+ *       aligned: t as [M, 64] bf16, then the fp32 partial sums of the down
+ *       projection's K slices; no initialisation needed.
+ */
+size_t w4a4_lora_workspace_bytes(int64_t M, int64_t K);
+int w4a4_lora_add(const uint16_t* x, int64_t ldx, const uint16_t* A, const uint16_t* B, int r, float scale,
+                  uint16_t* y, int64_t ldy, int64_t M, int64_t N, int64_t K, void* workspace,
+                  size_t workspace_bytes, void* stream);
+
+/*
+ * The fused layer (w4a4_linear_fused, act = 0) followed by the Dynamic LoRA
+ * update of w4a4_lora_add on its output.  Arguments as for those two calls;
+ * the workspace holds both (w4a4_fused_lora_workspace_bytes(M, N, K) bytes,
+ * 256-byte aligned).  GELU inputs (act = 1) are not supported here.
+ */
+size_t w4a4_fused_lora_workspace_bytes(int64_t M, int64_t N, int64_t K);
+int w4a4_linear_fused_lora(const uint16_t* x, int64_t ldx, const int8_t* Wq, const float* sw,
+                           const uint16_t* bias, const uint16_t* A, const uint16_t* B, int r, float scale,
+                           uint16_t* y, int64_t ldy, int64_t M, int64_t N, int64_t K, int g,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Synchronise `stream`, then read and clear the device status word that
  * kernels set when a bounded wait expires.  Returns W4A4_OK,
  * W4A4_ERR_TIMEOUT, or W4A4_ERR_CUDA if the synchronisation failed.

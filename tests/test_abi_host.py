@@ -228,3 +228,31 @@ def test_debug_wait_limit_rejects_bad_values(lib):
     assert lib.w4a4_debug_set_wait_limit(-1) == 9
     assert lib.w4a4_debug_set_wait_limit(3_000_000_000) == 9
     assert lib.w4a4_debug_set_wait_limit(0) == 0       # the default (2 s)
+
+
+def test_lora_entries_reject_bad_arguments(lib):
+    f = lib.w4a4_lora_add
+    base = dict(x=FAKE, ldx=256, A=FAKE, B=FAKE, r=32, scale=1.0, y=FAKE, ldy=256, M=10, N=256, K=256,
+                ws=NULL, wsb=0, st=NULL)
+    call = lambda **kw: f(*({**base, **kw}).values())
+    assert call(A=NULL) == 1
+    assert call(r=24) == 2                 # r in {16, 32, 48, 64}
+    assert call(r=128) == 2
+    assert call(N=100) == 2
+    assert call(ldx=100) == 2
+    assert call(y=MISALIGNED) == 4
+    assert call(scale=float("nan")) == 9
+    g = lib.w4a4_linear_fused_lora
+    gb = dict(x=FAKE, ldx=256, wq=FAKE, sw=FAKE, bias=NULL, A=FAKE, B=FAKE, r=32, scale=1.0, y=FAKE, ldy=256,
+              M=10, N=256, K=256, g=128, ws=NULL, wsb=0, st=NULL)
+    gcall = lambda **kw: g(*({**gb, **kw}).values())
+    assert gcall(B=NULL) == 1
+    assert gcall(g=96) == 3
+    assert gcall(r=8) == 2
+    # [t: M x 64 bf16][partials: slices x M x 64 fp32]; 36 row tiles take 8 K slices
+    assert lib.w4a4_lora_workspace_bytes(4608, 3072) == 4608 * 128 + 8 * 4608 * 256
+    # one row tile: up to 32 slices, at least one 64-element chunk each (K = 256: 4 slices)
+    assert lib.w4a4_lora_workspace_bytes(3, 256) == 512 + 4 * 3 * 256
+    # 48 chunks over at most 32 slices: 2 chunks per slice, so 24 slices
+    assert lib.w4a4_lora_workspace_bytes(16, 3072) == 2048 + 24 * 16 * 256
+    assert lib.w4a4_fused_lora_workspace_bytes(16, 3072, 3072) == (16 * 1536 + 256) + lib.w4a4_lora_workspace_bytes(16, 3072)

@@ -413,7 +413,7 @@ def test_bounded_wait_reports_timeout_and_context_survives(cuda_lib):
 
 
 @pytest.mark.parametrize("kernel", ["quant_butterfly", "quant_tensor_core", "gemm_tc", "gemm_small_m",
-                                    "fused_square"])
+                                    "fused_square", "lora"])
 def test_product_kernel_waits_expire_and_context_survives(cuda_lib, kernel):
     """With a wait limit of a few nanoseconds the product kernels' waits on
     their copy rings, widened stages, accumulators and cluster peers expire
@@ -430,6 +430,10 @@ def test_product_kernel_waits_expire_and_context_survives(cuda_lib, kernel):
     Xq, sx = cuda_lib.quantize_activation(big, g)
     x16 = workloads.make_activation(16, 12288, seed=80).cuda()
     Xq16, sx16 = cuda_lib.quantize_activation(x16, g)
+    gen = torch.Generator().manual_seed(81)
+    A = (torch.randn(64, 3072, generator=gen) * 0.02).to(torch.bfloat16).cuda()
+    B = (torch.randn(3072, 64, generator=gen) * 0.02).to(torch.bfloat16).cuda()
+    ylora = torch.zeros(4608, 3072, dtype=torch.bfloat16, device="cuda")
     torch.cuda.synchronize()
     assert cuda_lib.last_device_error() == 0
     runs = {
@@ -438,6 +442,7 @@ def test_product_kernel_waits_expire_and_context_survives(cuda_lib, kernel):
         "gemm_tc": lambda: cuda_lib.linear(Xq[:1000].contiguous(), sx[:1000].contiguous(), Wq, sw),
         "gemm_small_m": lambda: cuda_lib.linear(Xq16, sx16, Wqk, swk),
         "fused_square": lambda: cuda_lib.linear_fused(big, Wq, sw, None, g),
+        "lora": lambda: cuda_lib.lora_add(big, A, B, 0.25, ylora),
     }
     if kernel == "gemm_small_m":
         assert cuda_lib.linear_kernel(16, 3072, 12288) == 1

@@ -48,6 +48,11 @@ SIGNATURES = {
     "w4a4_gemm_s32": (_I, [_P, _P, _P, _I64, _I64, _I64, _I64, _I, _P, _SZ, _P]),
     "w4a4_linear_fused_noalloc": (_I, [_P, _I64, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I, _I, _P]),
 
+    "w4a4_lora_workspace_bytes": (_SZ, [_I64, _I64]),
+    "w4a4_lora_add": (_I, [_P, _I64, _P, _P, _I, ctypes.c_float, _P, _I64, _I64, _I64, _I64, _P, _SZ, _P]),
+    "w4a4_fused_lora_workspace_bytes": (_SZ, [_I64, _I64, _I64]),
+    "w4a4_linear_fused_lora": (_I, [_P, _I64, _P, _P, _P, _P, _P, _I, ctypes.c_float, _P, _I64, _I64, _I64, _I64,
+                                    _I, _P, _SZ, _P]),
     "w4a4_last_device_error": (_I, [_P]),
     "w4a4_debug_wait_timeout": (_I, [_I64, _P]),
     "w4a4_debug_set_wait_limit": (_I, [_I64]),
@@ -280,6 +285,50 @@ def linear_fused_noalloc(x, Wq, sw, bias=None, g=128, act=0, out=None):
     _need_rows(y, torch.bfloat16, M, N, "out", x.device)
     _check(lib.w4a4_linear_fused_noalloc(_ptr(x), x.stride(0), _ptr(Wq), _ptr(sw), _ptr(bias), _ptr(y), y.stride(0),
                                          M, N, K, g, act, _stream(x)), "w4a4_linear_fused_noalloc")
+    return y
+
+
+def _check_lora(A, B, K, N, device):
+    _need_cuda(A, torch.bfloat16, "A")
+    _need_cuda(B, torch.bfloat16, "B")
+    if A.dim() != 2 or A.shape[1] != K or not A.is_contiguous() or A.device != device:
+        raise ValueError("A must be a contiguous [r, K] bf16 tensor on the activation's device")
+    r = A.shape[0]
+    if B.dim() != 2 or tuple(B.shape) != (N, r) or not B.is_contiguous() or B.device != device:
+        raise ValueError("B must be a contiguous [N, r] bf16 tensor on the activation's device")
+    return r
+
+
+def lora_add(x, A, B, scale, y):
+    """Dynamic LoRA update in place: y += scale * (x A^T) B^T (see
+    w4a4_lora_add; the rotated form of the pages equals it)."""
+    lib = load_library()
+    _need_cuda(x, torch.bfloat16, "x")
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be a 2-D tensor with a contiguous inner dimension")
+    M, K = x.shape
+    N = y.shape[1]
+    _need_rows(y, torch.bfloat16, M, N, "y", x.device)
+    r = _check_lora(A, B, K, N, x.device)
+    nbytes = lib.w4a4_lora_workspace_bytes(M, K)
+    ws = workspace(nbytes, x.device, "lora") if nbytes else None
+    _check(lib.w4a4_lora_add(_ptr(x), x.stride(0), _ptr(A), _ptr(B), r, float(scale), _ptr(y), y.stride(0),
+                             M, N, K, _ptr(ws), nbytes, _stream(x)), "w4a4_lora_add")
+    return y
+
+
+def linear_fused_lora(x, Wq, sw, bias, A, B, scale, g=128, out=None):
+    """The fused layer plus its Dynamic LoRA update (w4a4_linear_fused_lora)."""
+    lib = load_library()
+    M, K, N = _check_fused_operands(x, Wq, sw, bias)
+    r = _check_lora(A, B, K, N, x.device)
+    y = out if out is not None else torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
+    _need_rows(y, torch.bfloat16, M, N, "out", x.device)
+    nbytes = lib.w4a4_fused_lora_workspace_bytes(M, N, K)
+    ws = workspace(nbytes, x.device, "fused_lora") if nbytes else None
+    _check(lib.w4a4_linear_fused_lora(_ptr(x), x.stride(0), _ptr(Wq), _ptr(sw), _ptr(bias), _ptr(A), _ptr(B), r,
+                                      float(scale), _ptr(y), y.stride(0), M, N, K, g, _ptr(ws), nbytes,
+                                      _stream(x)), "w4a4_linear_fused_lora")
     return y
 
 

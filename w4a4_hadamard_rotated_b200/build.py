@@ -18,7 +18,7 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libw4a4.so")
-SOURCES = ["api.cu", "quant.cu", "quant_tc.cu", "gemm.cu", "gemm_legacy.cu", "smallm.cu", "gemv.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "quant.cu", "quant_tc.cu", "gemm.cu", "gemm_legacy.cu", "smallm.cu", "gemv.cu", "noalloc.cu", "lora.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

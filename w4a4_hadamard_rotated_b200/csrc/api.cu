@@ -112,6 +112,19 @@ int group_rows_map(CUtensorMap* map, const uint16_t* x, int64_t M, int64_t K, in
   return r == CUDA_SUCCESS ? W4A4_OK : W4A4_ERR_CUDA;
 }
 
+int tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, int64_t rows, int64_t cols,
+                  int64_t row_stride_bytes, int box_cols, int box_rows, CUtensorMapSwizzle swizzle) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return W4A4_ERR_CUDA;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_stride_bytes)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? W4A4_OK : W4A4_ERR_CUDA;
+}
+
 namespace {
 
 // 2-D map over a bf16 output [rows, cols] with row stride ld (elements), box
@@ -444,6 +457,74 @@ int w4a4_linear_fused(const uint16_t* x, int64_t ldx, const int8_t* Wq, const fl
   // whatever wrote the weights is complete when the GEMM kernel starts: the
   // weight-streaming kernels may begin reading them before their own wait.
   return run_linear(xq, sx, Wq, sw, bias, y, M, N, K, ldy, 0, path, s, 1);
+}
+
+// [t: M x 64 bf16][the K slices' partial sums: slices x M x 64 fp32]
+static size_t lora_t_bytes(int64_t M) { return round256(static_cast<size_t>(M) * kLoraMaxRank * 2); }
+
+size_t w4a4_lora_workspace_bytes(int64_t M, int64_t K) {
+  if (M <= 0 || K <= 0) return 0;
+  return lora_t_bytes(M) + static_cast<size_t>(lora_slices(M, K)) * static_cast<size_t>(M) * kLoraMaxRank * 4;
+}
+
+int w4a4_lora_add(const uint16_t* x, int64_t ldx, const uint16_t* A, const uint16_t* B, int r, float scale,
+                  uint16_t* y, int64_t ldy, int64_t M, int64_t N, int64_t K, void* workspace, size_t workspace_bytes,
+                  void* stream) {
+  if (A == nullptr || B == nullptr) return W4A4_ERR_NULL;
+  if (M != 0 && (x == nullptr || y == nullptr)) return W4A4_ERR_NULL;
+  if (r < 16 || r > kLoraMaxRank || r % 16 != 0) return W4A4_ERR_SHAPE;
+  if (M < 0 || M > (int64_t(1) << 26)) return W4A4_ERR_SHAPE;
+  if (N < 1 || N % 8 != 0 || N > (int64_t(1) << 24)) return W4A4_ERR_SHAPE;
+  if (K < 8 || K % 8 != 0 || K > (int64_t(1) << 20)) return W4A4_ERR_SHAPE;
+  if (ldx < K || ldy < N) return W4A4_ERR_SHAPE;
+  if (ldx % 8 != 0 || ldy % 8 != 0 || !aligned(x, 16) || !aligned(y, 16) || !aligned(A, 16) || !aligned(B, 16))
+    return W4A4_ERR_ALIGN;
+  if (!(scale == scale) || scale > 3.0e38f || scale < -3.0e38f) return W4A4_ERR_ARG;   // finite
+  DeviceInfo* dev = nullptr;
+  int st = current_device(&dev);
+  if (st != W4A4_OK) return st;
+  if (M == 0) return W4A4_OK;
+  if (workspace == nullptr || workspace_bytes < w4a4_lora_workspace_bytes(M, K) || !aligned(workspace, 256))
+    return W4A4_ERR_WORKSPACE;
+  uint16_t* t = static_cast<uint16_t*>(workspace);
+  float* partial = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + lora_t_bytes(M));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (lora_down_launch(x, ldx, A, partial, t, M, K, r, dev->status, s) != cudaSuccess) return W4A4_ERR_CUDA;
+  return lora_up_launch(t, B, y, ldy, M, N, r, scale, dev->num_sms, dev->status, s) == cudaSuccess ? W4A4_OK
+                                                                                                   : W4A4_ERR_CUDA;
+}
+
+size_t w4a4_fused_lora_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  return w4a4_fused_workspace_bytes(M, N, K) + w4a4_lora_workspace_bytes(M, K);
+}
+
+int w4a4_linear_fused_lora(const uint16_t* x, int64_t ldx, const int8_t* Wq, const float* sw, const uint16_t* bias,
+                           const uint16_t* A, const uint16_t* B, int r, float scale, uint16_t* y, int64_t ldy,
+                           int64_t M, int64_t N, int64_t K, int g, void* workspace, size_t workspace_bytes,
+                           void* stream) {
+  int st = validate_fused(x, ldx, Wq, sw, bias, y, ldy, M, N, K, g, 0);
+  if (st != W4A4_OK) return st;
+  if (A == nullptr || B == nullptr) return W4A4_ERR_NULL;
+  if (r < 16 || r > kLoraMaxRank || r % 16 != 0) return W4A4_ERR_SHAPE;
+  if (!aligned(A, 16) || !aligned(B, 16)) return W4A4_ERR_ALIGN;
+  if (!(scale == scale) || scale > 3.0e38f || scale < -3.0e38f) return W4A4_ERR_ARG;
+  DeviceInfo* dev = nullptr;
+  if ((st = current_device(&dev)) != W4A4_OK) return st;
+  if (M == 0) return W4A4_OK;
+  const size_t base = w4a4_fused_workspace_bytes(M, N, K);
+  if (workspace == nullptr || workspace_bytes < base + w4a4_lora_workspace_bytes(M, K) || !aligned(workspace, 256))
+    return W4A4_ERR_WORKSPACE;
+  uint16_t* t = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(workspace) + base);
+  float* partial = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + base + lora_t_bytes(M));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // The down projection runs first, while x is still in L2 from the
+  // activation kernel of the previous layer call or its producer, then the
+  // fused layer, then the up projection adds to the layer's output.
+  if (lora_down_launch(x, ldx, A, partial, t, M, K, r, dev->status, s) != cudaSuccess) return W4A4_ERR_CUDA;
+  if ((st = w4a4_linear_fused(x, ldx, Wq, sw, bias, y, ldy, M, N, K, g, 0, workspace, base, stream)) != W4A4_OK)
+    return st;
+  return lora_up_launch(t, B, y, ldy, M, N, r, scale, dev->num_sms, dev->status, s) == cudaSuccess ? W4A4_OK
+                                                                                                   : W4A4_ERR_CUDA;
 }
 
 int w4a4_last_device_error(void* stream) {

@@ -108,6 +108,23 @@ cudaError_t smallm_launch_tm(const CUtensorMap& tmW, const CUtensorMap& tmX, con
 int smallm_rows_padded(int64_t M);
 constexpr int kSmallMMax = 64;
 
+// ---- Dynamic LoRA (lora.cu)
+// Largest LoRA rank; t is stored as [M, 64] bf16 (row stride 64, zero beyond r).
+constexpr int kLoraMaxRank = 64;
+// t[M, r] = x[M, K] A[r, K]^T (bf16 in, fp32 accumulation, bf16 out); the K
+// slices' fp32 partial sums go through `partial` (lora_slices(M, K) x M x 64
+// floats).
+int lora_slices(int64_t M, int64_t K);
+cudaError_t lora_down_launch(const uint16_t* x, int64_t ldx, const uint16_t* A, float* partial, uint16_t* t,
+                             int64_t M, int64_t K, int r, unsigned int* status, cudaStream_t stream);
+// y[M, N] = bf16(y + scale * t B^T), B [N, r] bf16.
+cudaError_t lora_up_launch(const uint16_t* t, const uint16_t* B, uint16_t* y, int64_t ldy, int64_t M, int64_t N,
+                           int r, float scale, int num_sms, unsigned int* status, cudaStream_t stream);
+// Generic 2-D TMA map: [rows, cols] elements, row stride in bytes, box
+// {box_cols, box_rows}; out-of-range elements read as zero.
+int tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, int64_t rows, int64_t cols,
+                  int64_t row_stride_bytes, int box_cols, int box_rows, CUtensorMapSwizzle swizzle);
+
 // ---- tiny-M weight streaming on the CUDA cores (gemv.cu)
 struct GemvArgs {
   const int8_t* xq;       // [M, K/2]
