@@ -125,11 +125,14 @@ __global__ void __launch_bounds__(kDownThreads)
       int issued = 0;
       for (int i = 0; i < nch; ++i) {
         const int s = i % kDownStages;
+        // row tiles start at different chunks of the slice, so that the CTAs
+        // of one slice do not all read the same chunk of A at once
+        const int c = c0 + (i + tile) % nch;
         if (!mbar_wait(&bars.empty[s], ((i / kDownStages) & 1) ^ 1, abort_flag, status, wait_ns)) break;
         mbar_arrive_expect_tx(&bars.full[s], kDownX + a_bytes);
         uint8_t* st = smem + s * kDownStage;
-        tma_load_2d(st, &tmX, &bars.full[s], (c0 + i) * kChunk, tile * kRows);
-        tma_load_2d(st + kDownX, &tmA, &bars.full[s], (c0 + i) * kChunk, 0);
+        tma_load_2d(st, &tmX, &bars.full[s], c * kChunk, tile * kRows);
+        tma_load_2d(st + kDownX, &tmA, &bars.full[s], c * kChunk, 0);
         ++issued;
       }
       // every issued copy lands before the ring is reused or the CTA exits
@@ -319,10 +322,12 @@ __global__ void __launch_bounds__(kUpThreads)
     }
   } else {
     // epilogue: warp w reads tensor-memory lanes 32 (w % 4) .. + 31 (= rows)
-    // and the half (w - 2) / 4 of the tile's columns.  The row's y values of
-    // the warp's 128 columns (16 x 16 bytes per lane) are loaded before the
-    // wait for the accumulator, so their latency overlaps the MMAs and the
-    // previous tile's tail.
+    // and the half (w - 2) / 4 of the tile's columns.  y is read and written
+    // through the same pointer, so loads of a later chunk would not be hoisted
+    // above the stores of an earlier one: the row's y values of all the
+    // warp's 128 columns (16 x 16 bytes per lane) are loaded first, before the
+    // wait for the accumulator, so that one memory latency per tile overlaps
+    // the MMAs instead of one per chunk in sequence.
     const int q = warp & 3;
     const int half = (warp - 2) / 4;
     const uint32_t tl = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
