@@ -117,3 +117,21 @@ def test_lora_down_projection_rows_are_independent(cuda_lib):
         yy = torch.zeros(m1 - m0, N, dtype=torch.bfloat16, device="cuda")
         cuda_lib.lora_add(x[m0:m1].contiguous(), A.cuda(), B.cuda(), 0.5, yy)
         assert torch.equal(yy.view(torch.int16), y[m0:m1].view(torch.int16))
+
+
+@pytest.mark.parametrize("M,N", [(200, 264), (129, 8)])
+def test_lora_into_a_strided_y_keeps_the_padding(cuda_lib, M, N):
+    """y with a row stride above N (a column slice of a wider buffer): the
+    update lands in the N columns only, equal to the update of a compact y,
+    and the padding columns keep their values."""
+    K, r = 1024, 32
+    x = workloads.make_activation(M, K, seed=11).cuda()
+    A, B = _lora_inputs(N, K, r, seed=12)
+    wide = workloads.make_activation(M, N + 72, seed=13).cuda()
+    pad0 = wide[:, N:].clone()
+    compact = wide[:, :N].clone()
+    cuda_lib.lora_add(x, A.cuda(), B.cuda(), 0.75, wide[:, :N])
+    cuda_lib.lora_add(x, A.cuda(), B.cuda(), 0.75, compact)
+    assert torch.equal(wide[:, :N].view(torch.int16), compact.view(torch.int16))
+    assert torch.equal(wide[:, N:].view(torch.int16), pad0.view(torch.int16))
+    assert cuda_lib.last_device_error() == 0

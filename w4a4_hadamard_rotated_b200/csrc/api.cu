@@ -517,12 +517,19 @@ int w4a4_linear_fused_lora(const uint16_t* x, int64_t ldx, const int8_t* Wq, con
   uint16_t* t = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(workspace) + base);
   float* partial = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + base + lora_t_bytes(M));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // The down projection runs first, while x is still in L2 from the
-  // activation kernel of the previous layer call or its producer, then the
-  // fused layer, then the up projection adds to the layer's output.
+  // The activation kernel reads x first; the down projection follows while
+  // x is still in L2; then the GEMM (its packed activation and scales from the
+  // workspace, as in w4a4_linear_fused) and the up projection, which adds to
+  // the layer's output.
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int8_t* xq = reinterpret_cast<int8_t*>(ws);
+  float* sx = reinterpret_cast<float*>(ws + fused_codes_bytes(M, K));
+  if ((st = w4a4_quantize_activation(x, M, K, ldx, g, 0, xq, sx, stream)) != W4A4_OK) return st;
   if (lora_down_launch(x, ldx, A, partial, t, M, K, r, dev->status, s) != cudaSuccess) return W4A4_ERR_CUDA;
-  if ((st = w4a4_linear_fused(x, ldx, Wq, sw, bias, y, ldy, M, N, K, g, 0, workspace, base, stream)) != W4A4_OK)
-    return st;
+  // every kernel before the GEMM has finished when it starts (the reduction
+  // kernel ahead of it completes before its dependents launch), so the
+  // weight-streaming kernels may read the weights before their own wait
+  if ((st = run_linear(xq, sx, Wq, sw, bias, y, M, N, K, ldy, 0, linear_path(M, K), s, 1)) != W4A4_OK) return st;
   return lora_up_launch(t, B, y, ldy, M, N, r, scale, dev->num_sms, dev->status, s) == cudaSuccess ? W4A4_OK
                                                                                                    : W4A4_ERR_CUDA;
 }

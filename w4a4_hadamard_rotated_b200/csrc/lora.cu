@@ -227,20 +227,23 @@ __global__ void __launch_bounds__(256)
 
 // ---------------------------------------------------------------- lora_up
 constexpr int kUpCols = 256;       // output columns per tile (MMA N)
-constexpr int kUpStages = 2;
+constexpr int kUpStages = 2;       // operand + y buffers
 constexpr int kUpEpiWarps = 8;     // two per tensor-memory lane quarter, one per half of the columns
 constexpr int kUpThreads = (2 + kUpEpiWarps) * 32;   // warp 0: TMA, warp 1: MMA, warps 2-9: epilogue
-constexpr uint32_t kUpT = kRows * 128;      // 16 KB
-constexpr uint32_t kUpB = kUpCols * 128;    // 32 KB
-constexpr uint32_t kUpStage = kUpT + kUpB;
-constexpr uint32_t kUpBytes = kUpStages * kUpStage;
+constexpr uint32_t kUpT = kRows * 128;      // 16 KB: t tile (128 rows x 64)
+constexpr uint32_t kUpB = kUpCols * 128;    // 32 KB: B tile (256 rows x 64)
+constexpr uint32_t kUpBox = kRows * 128;    // 16 KB: 64 columns x 128 rows of y (128-byte swizzle)
+constexpr uint32_t kUpY = 4 * kUpBox;       // 64 KB: the y tile (128 x 256), four boxes
+constexpr uint32_t kUpStage = kUpT + kUpB + kUpY;
+constexpr uint32_t kUpBytes = kUpStages * kUpStage;   // 224 KB
 constexpr uint32_t kUpAlloc = kUpBytes + 1024;
 
 struct UpBars {
-  uint64_t full[kUpStages];
-  uint64_t empty[kUpStages];
+  uint64_t full[kUpStages];     // t, B and y of a tile landed
+  uint64_t op_empty[kUpStages]; // the MMA has read t and B
+  uint64_t y_empty[kUpStages];  // the stores of the tile's y have read the buffer
   uint64_t acc_full;
-  uint64_t acc_empty;   // kUpEpiWarps epilogue warps
+  uint64_t acc_empty;           // kUpEpiWarps epilogue warps
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -248,7 +251,7 @@ struct UpBars {
 
 __global__ void __launch_bounds__(kUpThreads)
     lora_up_kernel(const __grid_constant__ CUtensorMap tmT, const __grid_constant__ CUtensorMap tmB,
-                   uint16_t* __restrict__ y, int64_t ldy, int64_t M, int64_t N, int r, float scale,
+                   const __grid_constant__ CUtensorMap tmY, int64_t M, int64_t N, int r, float scale,
                    unsigned int* status, unsigned long long wait_ns) {
   extern __shared__ uint8_t smem_dyn[];
   __shared__ UpBars bars;
@@ -262,7 +265,8 @@ __global__ void __launch_bounds__(kUpThreads)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kUpStages; ++s) {
       mbar_init(&bars.full[s], 1);
-      mbar_init(&bars.empty[s], 1);
+      mbar_init(&bars.op_empty[s], 1);
+      mbar_init(&bars.y_empty[s], 1);
     }
     mbar_init(&bars.acc_full, 1);
     mbar_init(&bars.acc_empty, kUpEpiWarps);
@@ -272,6 +276,7 @@ __global__ void __launch_bounds__(kUpThreads)
     fence_async_shared();
     tma_prefetch_desc(&tmT);
     tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmY);
   }
   if (warp == 1) {
     tmem_alloc(&bars.tmem_base, kUpCols);
@@ -286,23 +291,32 @@ __global__ void __launch_bounds__(kUpThreads)
   volatile int* abort_flag = &bars.abort_flag;
 
   if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
     if (lane == 0) {
       int issued = 0;
       for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++issued) {
         const int s = issued % kUpStages;
-        if (!mbar_wait(&bars.empty[s], ((issued / kUpStages) & 1) ^ 1, abort_flag, status, wait_ns)) break;
-        mbar_arrive_expect_tx(&bars.full[s], kUpStage);
+        const uint32_t par = ((issued / kUpStages) & 1) ^ 1;
+        if (!mbar_wait(&bars.op_empty[s], par, abort_flag, status, wait_ns) ||
+            !mbar_wait(&bars.y_empty[s], par, abort_flag, status, wait_ns))
+          break;
+        mbar_arrive_expect_tx(&bars.full[s], kUpT + kUpB + kUpY);
         uint8_t* st = smem + s * kUpStage;
         const int mb = t / num_n, nb = t % num_n;   // consecutive tiles of a CTA share the t tile
         tma_load_2d(st, &tmT, &bars.full[s], 0, mb * kRows);
         tma_load_2d(st + kUpT, &tmB, &bars.full[s], 0, nb * kUpCols);
+#pragma unroll
+        for (int b = 0; b < 4; ++b)
+          tma_load_2d(st + kUpT + kUpB + b * kUpBox, &tmY, &bars.full[s], nb * kUpCols + 64 * b, mb * kRows);
       }
+      // every issued copy lands before the CTA can exit
       for (int s = 0; s < kUpStages && s < issued; ++s) {
         const int n_s = issued / kUpStages + (s < issued % kUpStages ? 1 : 0);
         (void)mbar_wait(&bars.full[s], static_cast<uint32_t>((n_s - 1) & 1), nullptr, nullptr, 100000000ull);
       }
     }
   } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16(kRows, kUpCols);
       int i = 0;
@@ -314,52 +328,46 @@ __global__ void __launch_bounds__(kUpThreads)
         const uint64_t ad = sw128_kmajor_desc(smem_u32(smem + s * kUpStage));
         const uint64_t bd = sw128_kmajor_desc(smem_u32(smem + s * kUpStage + kUpT));
         for (int k = 0; k < r / 16; ++k) mma_bf16(tmem_base, ad + 2 * k, bd + 2 * k, idesc, k != 0 ? 1u : 0u);
-        mma_commit(&bars.empty[s]);
+        mma_commit(&bars.op_empty[s]);
         mma_commit(&bars.acc_full);
       }
       mma_commit(&bars.drain);
       (void)mbar_wait(&bars.drain, 0, nullptr, nullptr, 100000000ull);
     }
   } else {
-    // epilogue: warp w reads tensor-memory lanes 32 (w % 4) .. + 31 (= rows)
-    // and the half (w - 2) / 4 of the tile's columns.  y is read and written
-    // through the same pointer, so loads of a later chunk would not be hoisted
-    // above the stores of an earlier one: the row's y values of all the
-    // warp's 128 columns (16 x 16 bytes per lane) are loaded first, before the
-    // wait for the accumulator, so that one memory latency per tile overlaps
-    // the MMAs instead of one per chunk in sequence.
+    // ---------------------------------------------------------------- epilogue
+    // Warp w reads tensor-memory lanes 32 (w % 4) .. + 31 (= rows of the tile)
+    // and the half (w - 2) / 4 of its columns.  The tile's y arrived in shared
+    // memory by TMA (four 64-column boxes, 128-byte swizzle: 16-byte chunk c
+    // of row m at chunk c ^ (m & 7)); each thread adds scale * delta to its
+    // row's values in place, and one thread stores the boxes with TMA, which
+    // also clips the M and N tails.
     const int q = warp & 3;
     const int half = (warp - 2) / 4;
+    const int row = q * 32 + lane;
     const uint32_t tl = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-    constexpr int kCh = kUpCols / 2 / 32;   // 32-column chunks per warp
     int i = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
-      const int mb = t / num_n, nb = t % num_n;
-      const int64_t m = static_cast<int64_t>(mb) * kRows + q * 32 + lane;
-      const int64_t nw = static_cast<int64_t>(nb) * kUpCols + half * (kUpCols / 2);
-      uint16_t* yr = y + (m < M ? m * ldy : 0);
-      uint4 w[kCh][4];
-#pragma unroll
-      for (int ch = 0; ch < kCh; ++ch)
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int64_t n = nw + 32 * ch + 8 * u;
-          w[ch][u] = (m < M && n < N) ? *reinterpret_cast<const uint4*>(yr + n) : make_uint4(0u, 0u, 0u, 0u);
-        }
-      const bool ok = warp_wait(&bars.acc_full, i & 1, abort_flag, status, wait_ns);
-      if (!ok) break;   // nothing to drain: every later wait of this warp would fail too
+      const int s = i % kUpStages;
+      bool ok = warp_wait(&bars.full[s], (i / kUpStages) & 1, abort_flag, status, wait_ns) &&
+                warp_wait(&bars.acc_full, i & 1, abort_flag, status, wait_ns);
+      // one verdict for the eight warps: they meet named barriers below
+      if (bar_sync_or(1, kUpEpiWarps * 32, !ok)) break;
       tc_fence_after();
-#pragma unroll
-      for (int ch = 0; ch < kCh; ++ch) {
+      const uint32_t ybuf = smem_u32(smem + s * kUpStage + kUpT + kUpB);
+#pragma unroll 1
+      for (int ch = 0; ch < 4; ++ch) {
+        const int c = half * (kUpCols / 2) + 32 * ch;   // first column of the chunk in the tile
         uint32_t v[32];
-        tmem_ld_32x32b_x32(tl + half * (kUpCols / 2) + 32 * ch, v);
+        tmem_ld_32x32b_x32(tl + c, v);
         tmem_wait_ld();
-        if (m >= M) continue;
+        const uint32_t box = ybuf + (c / 64) * kUpBox + (row >> 3) * 1024 + (row & 7) * 128;
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          const int64_t n = nw + 32 * ch + 8 * u;
-          if (n >= N) break;   // N % 8 == 0: whole 16-byte units
-          uint32_t* wp = reinterpret_cast<uint32_t*>(&w[ch][u]);
+          const int cc = ((c % 64) / 8) + u;   // 16-byte chunk within the 128-byte box row
+          const uint32_t a = box + ((cc ^ (row & 7)) << 4);
+          uint4 w = lds128(a);
+          uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             // y + scale * delta with one rounding (a fused multiply-add), then bf16
@@ -368,13 +376,28 @@ __global__ void __launch_bounds__(kUpThreads)
                 __fmaf_rn(scale, __uint_as_float(v[8 * u + 2 * e + 1]), __uint_as_float(wp[e] & 0xFFFF0000u));
             wp[e] = pack_bf16x2(lo, hi);
           }
-          *reinterpret_cast<uint4*>(yr + n) = w[ch][u];
+          sts128(a, w);
         }
       }
       tc_fence_before();
+      fence_async_shared();   // the updated y is read next by the TMA stores
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.acc_empty);
+      if (lane == 0) mbar_arrive(&bars.acc_empty);   // the accumulator is free for the next tile
+      asm volatile("bar.sync 2, %0;" ::"n"(kUpEpiWarps * 32) : "memory");
+      if (warp == 2 && lane == 0) {
+        const int mb = t / num_n, nb = t % num_n;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          const int64_t n0 = static_cast<int64_t>(nb) * kUpCols + 64 * b;
+          if (n0 < N) tma_store_2d(&tmY, smem + s * kUpStage + kUpT + kUpB + b * kUpBox, static_cast<int32_t>(n0),
+                                   mb * kRows);
+        }
+        bulk_commit_group();
+        bulk_wait_group_read<0>();   // the stores have read the buffer
+        mbar_arrive(&bars.y_empty[s]);
+      }
     }
+    if (warp == 2 && lane == 0) bulk_wait_group_read<0>();
   }
   tc_fence_before();
   __syncthreads();
@@ -460,8 +483,9 @@ cudaError_t lora_down_launch(const uint16_t* x, int64_t ldx, const uint16_t* A, 
 
 cudaError_t lora_up_launch(const uint16_t* t, const uint16_t* B, uint16_t* y, int64_t ldy, int64_t M, int64_t N,
                            int r, float scale, int num_sms, unsigned int* status, cudaStream_t stream) {
-  CUtensorMap tmT, tmB;
-  if (bf16_map(&tmT, t, M, kLoraMaxRank, kLoraMaxRank, kRows) != 0 || bf16_map(&tmB, B, N, r, r, kUpCols) != 0)
+  CUtensorMap tmT, tmB, tmY;
+  if (bf16_map(&tmT, t, M, kLoraMaxRank, kLoraMaxRank, kRows) != 0 || bf16_map(&tmB, B, N, r, r, kUpCols) != 0 ||
+      bf16_map(&tmY, y, M, N, ldy, kRows) != 0)
     return cudaErrorInvalidValue;
   static bool attr_set[64] = {};
   int dev = 0;
@@ -469,16 +493,15 @@ cudaError_t lora_up_launch(const uint16_t* t, const uint16_t* B, uint16_t* y, in
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!attr_set[dev]) {
-    // (the default carve-out: a larger L1 serves the half-sector y accesses of
-    // the epilogue; the whole array as shared memory measured slower)
     e = cudaFuncSetAttribute(lora_up_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kUpAlloc);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(lora_up_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
   const int64_t tiles = ((M + kRows - 1) / kRows) * ((N + kUpCols - 1) / kUpCols);
-  // one CTA per SM: the epilogue's prefetched rows of y take about 110
-  // registers per thread, so two CTAs do not fit an SM's register file
-  const int64_t cap = static_cast<int64_t>(num_sms);
+  const int64_t cap = static_cast<int64_t>(num_sms);   // one CTA per SM (224 KB of shared memory)
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(tiles < cap ? tiles : cap), 1, 1);
   cfg.blockDim = dim3(kUpThreads, 1, 1);
@@ -489,7 +512,7 @@ cudaError_t lora_up_launch(const uint16_t* t, const uint16_t* B, uint16_t* y, in
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, lora_up_kernel, tmT, tmB, y, ldy, M, N, r, scale, status, wait_limit_ns());
+  e = cudaLaunchKernelEx(&cfg, lora_up_kernel, tmT, tmB, tmY, M, N, r, scale, status, wait_limit_ns());
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
