@@ -21,13 +21,14 @@
 //     order (deterministic) and stores t in bf16 with a row stride of 64
 //     elements, zero beyond r.  (Reducing the slices on chip, within a CTA
 //     cluster, measured slower: only 15 clusters of eight fit at once.)
-//   * lora_up: y[M, N] = bf16(y + scale * t B^T).  A persistent CTA takes
-//     128 x 256 output tiles: TMA loads the t tile (128 x 64) and the B tile
-//     (256 x 64, zero beyond r), one thread issues r / 16 MMAs (M = 128,
+//   * lora_up: y[M, N] = bf16(y + scale * t B^T).  A persistent CTA (one
+//     per SM) takes 128 x 256 output tiles: TMA loads the t tile (128 x 64),
+//     the B tile (256 x 64, zero beyond r) and the y tile (four 64-column
+//     boxes) into one of two stages, one thread issues r / 16 MMAs (M = 128,
 //     N = 256, K = 16) into 256 fp32 columns of tensor memory, and eight
-//     epilogue warps (two per lane quarter, one per half of the columns) read
-//     each row's 32-column chunks back, add scale * delta to the bf16 y in
-//     fp32 and store y rounded to bf16.
+//     epilogue warps (two per lane quarter, one per half of the columns) add
+//     scale * delta to the staged y in place; one thread then writes the
+//     boxes back with TMA stores, which clip the M and N tails.
 //   Every wait is bounded; an expired wait records W4A4_ERR_TIMEOUT, every
 //   role stops, copies and MMAs drain and tensor memory is freed.
 #include <cuda_bf16.h>

@@ -557,8 +557,9 @@ static cudaError_t dispatch_rq(const TIn* x, int64_t M, int K, int64_t ldx, int 
 // but inside the fused layer, ahead of the GEMM, only the 32760-row shapes
 // gain (0.7%) while 4608-row layers lose 1-2 us, so by default it serves
 // batches of 8192 rows and more.  W4A4_ROTATE_TC_MIN_ROWS=<n> moves the
-// threshold (the test suite sets 512 so that its parity cases reach both
-// kernels); W4A4_ROTATE_TC=0 selects the register-butterfly kernel always.
+// threshold and W4A4_ROTATE_TC=0 selects the register-butterfly kernel
+// always (both read once per process); w4a4_quantize_activation_path picks a
+// kernel per call.
 static int64_t rotate_tc_min_rows() {
   static int64_t v = -1;
   static std::once_flag once;
