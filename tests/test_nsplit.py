@@ -109,12 +109,23 @@ def test_column_blocks_on_the_gpu_match_the_whole_layer(cuda_lib, M, K, N, world
     Wq, sw = cuda_lib.quantize_weight(W.cuda(), cfg.g)
     bc = b.cuda()
     whole = cuda_lib.linear_fused(xc, Wq, sw, bc, cfg.g)
-    for rank, (a, e) in enumerate(nsplit.column_blocks(N, world)):
+    blocks = nsplit.column_blocks(N, world)
+    width = max(e - a for a, e in blocks)
+    # what the ranks send: each block written by the layer straight into a
+    # zeroed [M, width] buffer (row stride width), as NSplitLinear does
+    sends = torch.zeros(world, M, width, dtype=torch.bfloat16, device="cuda")
+    for rank, (a, e) in enumerate(blocks):
         if e == a:
             continue
         Wq_r, sw_r, b_r = nsplit.shard_weight(Wq, sw, bc, world, rank)
         y_r = cuda_lib.linear_fused(xc, Wq_r, sw_r, b_r, cfg.g)
         assert torch.equal(y_r.view(torch.int16), whole[:, a:e].contiguous().view(torch.int16))
+        cuda_lib.linear_fused(xc, Wq_r, sw_r, b_r, cfg.g, out=sends[rank, :, : e - a])
+        assert torch.equal(sends[rank, :, : e - a].view(torch.int16), y_r.view(torch.int16))
+        assert not sends[rank, :, e - a:].view(torch.int16).any()   # padding untouched
+    # the all-gather's result is the sends stacked along rows; placing it gives y
+    y = nsplit._place_blocks(sends.view(world * M, width), torch.empty_like(whole), blocks, M, width)
+    assert torch.equal(y.view(torch.int16), whole.view(torch.int16))
     # world = 1 (no process group): the split layer is the whole layer
     y = nsplit.NSplitLinear(Wq, sw, bc, cfg.g)(xc)
     assert torch.equal(y.view(torch.int16), whole.view(torch.int16))

@@ -49,6 +49,22 @@ def shard_weight(Wq, sw, bias, world, rank):
     return Wq[n0:n1], sw[n0:n1], (bias[n0:n1] if bias is not None else None)
 
 
+def _place_blocks(recv, out, blocks, M, width):
+    """Copy the gathered blocks (recv viewed as [world, M, width]) into their
+    column slices of out [M, N]: one strided copy when every block is
+    `width` wide and out is contiguous, else one copy per block."""
+    world = len(blocks)
+    N = blocks[-1][1]
+    r3 = recv.view(world, M, width)
+    if N == world * width and out.is_contiguous():
+        out.view(M, world, width).copy_(r3.permute(1, 0, 2))
+        return out
+    for r, (a, b) in enumerate(blocks):
+        if b > a:
+            out[:, a:b].copy_(r3[r, :, : b - a])
+    return out
+
+
 def gather_columns(y_local, N, world, rank, group=None, out=None):
     """All-gather the ranks' column blocks into the full y [M, N].
 
@@ -71,13 +87,9 @@ def gather_columns(y_local, N, world, rank, group=None, out=None):
         dist.all_gather_into_tensor(recv, send, group=group)
     else:
         recv.copy_(send)
-    recv = recv.view(world, M, width)
     if out is None:
         out = torch.empty(M, N, dtype=y_local.dtype, device=y_local.device)
-    for r, (a, b) in enumerate(blocks):
-        if b > a:
-            out[:, a:b].copy_(recv[r, :, : b - a])
-    return out
+    return _place_blocks(recv, out, blocks, M, width)
 
 
 class NSplitLinear:
@@ -86,7 +98,13 @@ class NSplitLinear:
     [N, K/2], sw [N], bias [N] or None; each rank keeps only its block) or
     with `pre_sharded=True` and this rank's block.  Calling it with the
     activation x [M, K] (bf16, the same on every rank) returns the full
-    y [M, N] on every rank."""
+    y [M, N] on every rank.
+
+    Each rank writes its block of y straight into its all-gather send buffer
+    (a row stride of the widest block), and the send and receive buffers are
+    kept per batch size and device, so a call allocates nothing after the
+    first one of its shape (besides `out`, when not given).  With one rank
+    the layer writes y directly."""
 
     def __init__(self, Wq, sw, bias=None, g=128, group=None, pre_sharded=False, N=None):
         import torch.distributed as dist
@@ -106,13 +124,31 @@ class NSplitLinear:
         else:
             self.N = Wq.shape[0]
             self.Wq, self.sw, self.bias = shard_weight(Wq, sw, bias, self.world, self.rank)
+        self.blocks = column_blocks(self.N, self.world)
+        self.width = max(b - a for a, b in self.blocks)
+        self._bufs = {}
+
+    def _buffers(self, M, device):
+        key = (M, device)
+        if key not in self._bufs:
+            # padding columns of send are never written: they stay zero
+            send = torch.zeros(M, self.width, dtype=torch.bfloat16, device=device)
+            recv = torch.empty(self.world * M, self.width, dtype=torch.bfloat16, device=device)
+            self._bufs[key] = (send, recv)
+        return self._bufs[key]
 
     def __call__(self, x, act=0, out=None):
+        import torch.distributed as dist
         from . import linear_fused
 
         M = x.shape[0]
-        if self.Wq.shape[0] > 0:
-            y_local = linear_fused(x, self.Wq, self.sw, self.bias, self.g, act)
-        else:
-            y_local = torch.empty(M, 0, dtype=torch.bfloat16, device=x.device)
-        return gather_columns(y_local, self.N, self.world, self.rank, self.group, out)
+        if self.world == 1:
+            return linear_fused(x, self.Wq, self.sw, self.bias, self.g, act, out=out)
+        n0, n1 = self.blocks[self.rank]
+        send, recv = self._buffers(M, x.device)
+        if n1 > n0:
+            linear_fused(x, self.Wq, self.sw, self.bias, self.g, act, out=send[:, : n1 - n0])
+        dist.all_gather_into_tensor(recv, send, group=self.group)
+        if out is None:
+            out = torch.empty(M, self.N, dtype=torch.bfloat16, device=x.device)
+        return _place_blocks(recv, out, self.blocks, M, self.width)
