@@ -240,7 +240,8 @@ constexpr uint32_t kUpBytes = kUpStages * kUpStage;   // 224 KB
 constexpr uint32_t kUpAlloc = kUpBytes + 1024;
 
 struct UpBars {
-  uint64_t full[kUpStages];     // t, B and y of a tile landed
+  uint64_t full[kUpStages];     // t and B of a tile landed
+  uint64_t yfull[kUpStages];    // the tile's y landed
   uint64_t op_empty[kUpStages]; // the MMA has read t and B
   uint64_t y_empty[kUpStages];  // the stores of the tile's y have read the buffer
   uint64_t acc_full;
@@ -266,6 +267,7 @@ __global__ void __launch_bounds__(kUpThreads)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kUpStages; ++s) {
       mbar_init(&bars.full[s], 1);
+      mbar_init(&bars.yfull[s], 1);
       mbar_init(&bars.op_empty[s], 1);
       mbar_init(&bars.y_empty[s], 1);
     }
@@ -301,19 +303,25 @@ __global__ void __launch_bounds__(kUpThreads)
         if (!mbar_wait(&bars.op_empty[s], par, abort_flag, status, wait_ns) ||
             !mbar_wait(&bars.y_empty[s], par, abort_flag, status, wait_ns))
           break;
-        mbar_arrive_expect_tx(&bars.full[s], kUpT + kUpB + kUpY);
+        // t and B (the MMA's operands) on one barrier, y on another, so that
+        // the MMA need not wait for y; y boxes wholly past N are not loaded
+        // (the epilogue stores none of them either)
+        mbar_arrive_expect_tx(&bars.full[s], kUpT + kUpB);
         uint8_t* st = smem + s * kUpStage;
-        const int mb = t / num_n, nb = t % num_n;   // consecutive tiles of a CTA share the t tile
+        const int mb = t / num_n, nb = t % num_n;   // CTAs running side by side share t and B tiles in L2
         tma_load_2d(st, &tmT, &bars.full[s], 0, mb * kRows);
         tma_load_2d(st + kUpT, &tmB, &bars.full[s], 0, nb * kUpCols);
-#pragma unroll
-        for (int b = 0; b < 4; ++b)
-          tma_load_2d(st + kUpT + kUpB + b * kUpBox, &tmY, &bars.full[s], nb * kUpCols + 64 * b, mb * kRows);
+        const int64_t nrem = N - static_cast<int64_t>(nb) * kUpCols;
+        const int boxes = nrem >= kUpCols ? 4 : static_cast<int>((nrem + 63) / 64);
+        mbar_arrive_expect_tx(&bars.yfull[s], static_cast<uint32_t>(boxes) * kUpBox);
+        for (int b = 0; b < boxes; ++b)
+          tma_load_2d(st + kUpT + kUpB + b * kUpBox, &tmY, &bars.yfull[s], nb * kUpCols + 64 * b, mb * kRows);
       }
       // every issued copy lands before the CTA can exit
       for (int s = 0; s < kUpStages && s < issued; ++s) {
         const int n_s = issued / kUpStages + (s < issued % kUpStages ? 1 : 0);
         (void)mbar_wait(&bars.full[s], static_cast<uint32_t>((n_s - 1) & 1), nullptr, nullptr, 100000000ull);
+        (void)mbar_wait(&bars.yfull[s], static_cast<uint32_t>((n_s - 1) & 1), nullptr, nullptr, 100000000ull);
       }
     }
   } else if (warp == 1) {
@@ -350,7 +358,7 @@ __global__ void __launch_bounds__(kUpThreads)
     int i = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
       const int s = i % kUpStages;
-      bool ok = warp_wait(&bars.full[s], (i / kUpStages) & 1, abort_flag, status, wait_ns) &&
+      bool ok = warp_wait(&bars.yfull[s], (i / kUpStages) & 1, abort_flag, status, wait_ns) &&
                 warp_wait(&bars.acc_full, i & 1, abort_flag, status, wait_ns);
       // one verdict for the eight warps: they meet named barriers below
       if (bar_sync_or(1, kUpEpiWarps * 32, !ok)) break;
