@@ -46,4 +46,6 @@ from .w4a4_oracle import (  # noqa: F401
     boundary_window,
     lora_delta,
     linear_lora,
+    requant_partials,
+    chain_requant,
 )

@@ -276,3 +276,50 @@ def linear_lora(x_bits, wq_packed, sw, bias_bits, g, A, B, scale, act=0):
     out = dict(base)
     out.update({"t": t, "delta": delta, "base_y32": base["y32"], "y32": y32, "y_bits": f32_to_bf16_bits(y32)})
     return out
+
+
+# ---------------------------------------------------------------------------
+# Layer chains.  The down layer of an MLP quantises GELU of the up layer's
+# bf16 output (the pages' activation pass -- page "[PR #63] int4_tensorwise:
+# W4A4 layout (+ConvRot) with fused CUDA kernels", Description: rotate, then
+# one int4 scale per row -- applied to that output).  A requantising epilogue
+# splits it in two: the producing layer's column tiles each report, per row,
+# the amax of the rotated values in their columns; the row scale is the max
+# of those over the row, divided by 7, and the codes follow from it.
+# ---------------------------------------------------------------------------
+
+
+def requant_partials(y_bits, g, block_cols, act=1):
+    """Per-row amax of the rotated next-layer activation r = rotate(GELU(y))
+    (GELU only for act = 1) over each block of `block_cols` consecutive
+    columns (a multiple of g, so that no rotation group straddles blocks;
+    the last block may be narrower).  float32 [R, ceil(K / block_cols)]."""
+    if block_cols % g != 0:
+        raise ValueError("column blocks must hold whole rotation groups")
+    xf = bf16_bits_to_f32(y_bits)
+    if act == 1:
+        xf = gelu_f32(xf)
+    elif act != 0:
+        raise ValueError("act must be 0 (none) or 1 (gelu)")
+    _, r = rotate_rows(xf, g)
+    R, K = r.shape
+    nb = -(-K // block_cols)
+    out = np.zeros((R, nb), dtype=np.float32)
+    for b in range(nb):
+        out[:, b] = np.max(np.abs(r[:, b * block_cols:(b + 1) * block_cols]), axis=1)
+    return out
+
+
+def chain_requant(y_bits, g, block_cols, act=1):
+    """The next layer's packed codes and row scales from the producing
+    layer's bf16 output, by the two passes: the row amax as the max of the
+    block partials, s = amax / 7 (float32), codes = quantise(r / s).  Equal
+    to quantize_activation(y_bits, g, act) by construction (the max of the
+    block maxima is the row maximum); returned with the partials."""
+    parts = requant_partials(y_bits, g, block_cols, act)
+    amax = np.max(parts, axis=1).astype(np.float32)
+    out = dict(quantize_activation(y_bits, g, act))
+    out["partials"] = parts
+    out["amax"] = amax
+    out["scale_from_partials"] = (amax / np.float32(7.0)).astype(np.float32)
+    return out

@@ -451,3 +451,72 @@ def test_lora_with_gelu_input_uses_gelu_of_x():
     t1, _ = orc.lora_delta(xb, A, B, 64, 1.0, act=1)
     xg = orc.gelu_f32(orc.bf16_bits_to_f32(xb)).astype(np.float64)
     assert np.allclose(t1, xg @ A.astype(np.float64).T, rtol=1e-12, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# Layer chains: the requantising epilogue's two passes
+# --------------------------------------------------------------------------
+
+def test_requant_partials_hand_case():
+    """One nonzero input t per row, in different column blocks: after GELU
+    the rotation spreads G = GELU(t) over its 128-group as +-G / sqrt(128),
+    so that block's partial is fl(|G| / sqrt(128)) (the oracle rounds the
+    float64 sum u / sqrt(g) once), every other block's partial is 0, and the
+    row scale from the partials is that value / 7."""
+    g, bc, K = 128, 256, 768
+    ts = [1.25, -0.5, 3.0]
+    xb = np.zeros((3, K), dtype=np.uint16)
+    for i, (t, col) in enumerate(zip(ts, [5, 300, 767])):
+        xb[i, col] = orc.f32_to_bf16_bits(np.array([t], dtype=np.float32))[0]
+    parts = orc.requant_partials(xb, g, bc, act=1)
+    assert parts.shape == (3, 3)
+    for i, (t, col) in enumerate(zip(ts, [5, 300, 767])):
+        G = np.float64(np.float32(0.5 * t * (1.0 + math.erf(t / math.sqrt(2.0)))))
+        want = np.float32(abs(G) / math.sqrt(128.0))
+        for b in range(3):
+            assert parts[i, b] == (want if b == col // bc else 0.0)
+    out = orc.chain_requant(xb, g, bc, act=1)
+    assert np.array_equal(out["scale_from_partials"], out["scale"])
+
+
+def test_requant_partials_brute_force():
+    """Small random rows: every partial equals a loop over the block's
+    groups with scipy's dense Hadamard matrix and math.erf per element."""
+    import scipy.linalg
+    rng = np.random.default_rng(5)
+    g, bc, K, R = 64, 192, 448, 4     # the last block is 64 wide
+    x = (rng.standard_normal((R, K)) * 2).astype(np.float32)
+    xb = orc.f32_to_bf16_bits(x)
+    xf = orc.bf16_bits_to_f32(xb).astype(np.float64)
+    H = scipy.linalg.hadamard(g).astype(np.float64)
+    parts = orc.requant_partials(xb, g, bc, act=1)
+    assert parts.shape == (R, 3)
+    for m in range(R):
+        z = np.array([np.float32(0.5 * v * (1.0 + math.erf(v / math.sqrt(2.0)))) for v in xf[m]], dtype=np.float64)
+        for b in range(3):
+            best = 0.0
+            for k0 in range(b * bc, min(K, (b + 1) * bc), g):
+                r = (H @ z[k0:k0 + g]) / math.sqrt(g)
+                best = max(best, float(np.max(np.abs(r.astype(np.float32)))))
+            assert abs(parts[m, b] - best) <= 2e-7 * best
+
+
+@pytest.mark.parametrize("g,bc", [(64, 256), (128, 256), (256, 256), (128, 384)])
+def test_chain_requant_equals_the_layer_quantiser(g, bc):
+    """The two passes give exactly the one-pass quantisation of GELU(y):
+    the max of the block partials is the row amax, so the scales (and with
+    them the codes) agree bit for bit; and dropping a block's partial (a
+    tile that did not report) changes the scale of the rows whose maximum
+    sits in it."""
+    rng = np.random.default_rng(g + bc)
+    K = 1536
+    y = (rng.standard_normal((6, K)) * rng.uniform(0.2, 4.0, size=(6, 1))).astype(np.float32)
+    yb = orc.f32_to_bf16_bits(y)
+    out = orc.chain_requant(yb, g, bc, act=1)
+    assert np.array_equal(out["scale_from_partials"], out["scale"])
+    one = orc.quantize_activation(yb, g, act=1)
+    assert np.array_equal(out["packed"], one["packed"]) and np.array_equal(out["scale"], one["scale"])
+    arg = np.argmax(out["partials"], axis=1)
+    dropped = out["partials"].copy()
+    dropped[np.arange(6), arg] = 0.0
+    assert np.all(np.max(dropped, axis=1) < out["amax"])
