@@ -419,6 +419,55 @@ def measure_lora(w4, cfg, args, world, repeats, peaks, r=64):
                                      "kernels": "lora_down_kernel (t = x A^T) + lora_up_kernel (y += scale t B^T)"}}
 
 
+def measure_chain(w4, args, world, repeats):
+    """The MLP pair (up 4608x3072->12288, GELU, down 12288->3072) two ways,
+    each timed like a layer (CUDA-graph regions of exactly --steps pairs):
+    two fused layers (the down layer's activation kernel quantises GELU(y)),
+    and the up layer with the requantising epilogue
+    (w4a4_linear_fused_requant) feeding the down GEMM its codes directly."""
+    device = torch.device("cuda", torch.cuda.current_device())
+    up, down = workloads.MLP_UP, workloads.MLP_DOWN
+    sets = []
+    for i in range(3):
+        c = workloads.Linear(up.name, M=up.M, K=up.K, N=up.N, g=up.g, seed=up.seed + 100 * i)
+        x, W, b = c.make()
+        Wd = workloads.make_weight(down.N, down.K, seed=down.seed + 100 * i)
+        bd = workloads.make_bias(down.N, seed=down.seed + 100 * i + 1)
+        Wq, sw = w4.quantize_weight(W.to(device), up.g)
+        Wdq, swd = w4.quantize_weight(Wd.to(device), down.g)
+        sets.append({"x": x.to(device), "Wq": Wq, "sw": sw, "b": b.to(device), "Wdq": Wdq, "swd": swd,
+                     "bd": bd.to(device), "y": torch.empty(up.M, up.N, dtype=torch.bfloat16, device=device),
+                     "y2": torch.empty(up.M, down.N, dtype=torch.bfloat16, device=device),
+                     "xq": torch.empty(up.M, up.N // 2, dtype=torch.int8, device=device),
+                     "sx": torch.empty(up.M, dtype=torch.float32, device=device)})
+
+    def plain(i):
+        s = sets[i % 3]
+        w4.linear_fused(s["x"], s["Wq"], s["sw"], s["b"], up.g, 0, out=s["y"])
+        w4.linear_fused(s["y"], s["Wdq"], s["swd"], s["bd"], down.g, 1, out=s["y2"])
+
+    def chained(i):
+        s = sets[i % 3]
+        w4.linear_fused_requant(s["x"], s["Wq"], s["sw"], s["b"], up.g, 0, down.g, out=s["y"], xq_next=s["xq"],
+                                sx_next=s["sx"])
+        w4.linear(s["xq"], s["sx"], s["Wdq"], s["swd"], s["bd"], out=s["y2"])
+
+    out = {"workload": "mlp pair 4608x3072->12288 -> GELU -> 12288->3072 g128"}
+    for name, fn in (("two_fused_layers", plain), ("requant_epilogue", chained)):
+        for i in range(args.warmup):
+            fn(i)
+        torch.cuda.synchronize()
+        loop = GraphLoop(fn, args.steps)
+        loop.run()
+        per_step = [t / args.steps for t in time_regions(loop, repeats, world)]
+        del loop
+        out[name] = {"us_per_pair": statistics.median(per_step) * 1e6, "us_per_pair_min": min(per_step) * 1e6,
+                     "timed_regions": len(per_step)}
+    out["ops_per_pair"] = up.ops() + down.ops()
+    del sets
+    return out
+
+
 def layer_summary(w4, cfg, m, peaks):
     """The per-layer keys of the JSON line."""
     roof = layer_roofline_s(cfg, peaks)
@@ -522,6 +571,8 @@ def run_impl(args, cfg, world, rank, local):
 
     if args.workload == "square" and not args.no_extra_layers:
         extra["square_dynamic_lora_r64"] = measure_lora(w4, cfg, args, world, repeats, peaks)
+        torch.cuda.empty_cache()
+        extra["mlp_pair_chain"] = measure_chain(w4, args, world, repeats)
         torch.cuda.empty_cache()
 
     err = w4.last_device_error()

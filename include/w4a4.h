@@ -213,6 +213,41 @@ int w4a4_linear_fused_noalloc(const uint16_t* x, int64_t ldx, const int8_t* Wq, 
                               int g, int act, void* stream);
 
 /*
+ * Layer chains: the fused layer (w4a4_linear_fused) together with the
+ * quantised input of the layer after it, taken from GELU of this layer's
+ * output -- what w4a4_quantize_activation(y, M, N, ldy, g_next, act = 1, ...)
+ * returns (page "[PR #63] int4_tensorwise: W4A4 layout (+ConvRot) with fused
+ * CUDA kernels", Description: the activation pass -- rotate, one int4 scale
+ * per row, pack -- here applied to the layer's own output).  The row scale
+ * needs the amax of a whole output row, which many output tiles produce, so
+ * it runs in two passes: the GEMM's epilogue applies GELU and the rotation to
+ * every output tile it has just written and records, per row, the largest
+ * rotated magnitude over the tile's columns (atomic maxima in the
+ * workspace); a streaming kernel then rotates and quantises y with the row
+ * amax already known (no row reduction).  This entry has no counterpart in
+ * the pages, whose layers quantise their input in a pass of their own.
+ *   Arguments as for w4a4_linear_fused, plus:
+ *   g_next   rotation group of the next layer, in {64, 128, 256}; N is the
+ *            next layer's K: N % 128 == 0, N % g_next == 0, N <= 32768
+ *   Xq_next  [M, N / 2] packed int4 codes (16-byte aligned), written
+ *   sx_next  [M] fp32 row scales, written
+ *   workspace: w4a4_fused_requant_workspace_bytes(M, N, K) bytes, 256-byte
+ *       aligned (the activation codes of x, their scales and the row amax
+ *       slots; the call sets the slots to zero itself).
+ * y is bit-identical to w4a4_linear_fused's.  Xq_next and sx_next match the
+ * one-pass activation kernel up to the rounding of the rotated values (both
+ * passes form GELU with its table; the rotation is summed in another order).
+ * Batches that w4a4_linear_kernel routes to the
+ * weight-streaming kernels (M <= 64) run the layer and then the one-pass
+ * activation kernel on y.
+ */
+size_t w4a4_fused_requant_workspace_bytes(int64_t M, int64_t N, int64_t K);
+int w4a4_linear_fused_requant(const uint16_t* x, int64_t ldx, const int8_t* Wq, const float* sw,
+                              const uint16_t* bias, uint16_t* y, int64_t ldy, int64_t M, int64_t N, int64_t K,
+                              int g, int act, int g_next, int8_t* Xq_next, float* sx_next, void* workspace,
+                              size_t workspace_bytes, void* stream);
+
+/*
  * Dynamic LoRA (page "Comfy-INT4-HIPtest README", section "LoRA modes":
  * Dynamic keeps the LoRA matrices separate and applies their deltas at
  * inference time; page "ComfyUI-INT4-Fast", "Dynamic LoRA Patching": the

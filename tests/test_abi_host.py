@@ -256,3 +256,22 @@ def test_lora_entries_reject_bad_arguments(lib):
     # 48 chunks over at most 32 slices: 2 chunks per slice, so 24 slices
     assert lib.w4a4_lora_workspace_bytes(16, 3072) == 2048 + 24 * 16 * 256
     assert lib.w4a4_fused_lora_workspace_bytes(16, 3072, 3072) == (16 * 1536 + 256) + lib.w4a4_lora_workspace_bytes(16, 3072)
+
+
+def test_fused_requant_rejects_bad_arguments(lib):
+    f = lib.w4a4_linear_fused_requant
+    base = dict(x=FAKE, ldx=256, wq=FAKE, sw=FAKE, bias=NULL, y=FAKE, ldy=512, M=10, N=512, K=256, g=128, act=0,
+                g_next=128, xq=FAKE, sx=FAKE, ws=NULL, wsb=0, st=NULL)
+    call = lambda **kw: f(*({**base, **kw}).values())
+    assert call(xq=NULL) == 1
+    assert call(sx=NULL) == 1
+    assert call(g_next=96) == 3            # the next layer's group
+    assert call(N=384, ldy=384, g_next=256) == 3   # N % g_next
+    assert call(N=264, ldy=264) == 2       # N is the next layer's K: a multiple of 128
+    assert call(xq=MISALIGNED) == 4
+    assert call(g=96) == 3                 # this layer's own arguments as for w4a4_linear_fused
+    # [packed x][sx][row amax slots], each rounded up to 256 bytes
+    assert lib.w4a4_fused_requant_workspace_bytes(4608, 12288, 3072) == \
+        lib.w4a4_fused_workspace_bytes(4608, 12288, 3072) + 4608 * 4
+    assert lib.w4a4_fused_requant_workspace_bytes(3, 256, 256) == (512 + 256) + 256
+    assert lib.w4a4_fused_requant_workspace_bytes(0, 256, 256) == 0

@@ -53,6 +53,9 @@ SIGNATURES = {
     "w4a4_fused_lora_workspace_bytes": (_SZ, [_I64, _I64, _I64]),
     "w4a4_linear_fused_lora": (_I, [_P, _I64, _P, _P, _P, _P, _P, _I, ctypes.c_float, _P, _I64, _I64, _I64, _I64,
                                     _I, _P, _SZ, _P]),
+    "w4a4_fused_requant_workspace_bytes": (_SZ, [_I64, _I64, _I64]),
+    "w4a4_linear_fused_requant": (_I, [_P, _I64, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I, _I, _I, _P, _P, _P, _SZ,
+                                       _P]),
     "w4a4_last_device_error": (_I, [_P]),
     "w4a4_debug_wait_timeout": (_I, [_I64, _P]),
     "w4a4_debug_set_wait_limit": (_I, [_I64]),
@@ -315,6 +318,28 @@ def lora_add(x, A, B, scale, y):
     _check(lib.w4a4_lora_add(_ptr(x), x.stride(0), _ptr(A), _ptr(B), r, float(scale), _ptr(y), y.stride(0),
                              M, N, K, _ptr(ws), nbytes, _stream(x)), "w4a4_lora_add")
     return y
+
+
+def linear_fused_requant(x, Wq, sw, bias=None, g=128, act=0, g_next=128, out=None, xq_next=None, sx_next=None):
+    """The fused layer y = layer(x) together with the next layer's quantised
+    input from GELU(y) (w4a4_linear_fused_requant): returns (y [M, N] bf16,
+    Xq_next [M, N/2] int8, sx_next [M] fp32)."""
+    lib = load_library()
+    M, K, N = _check_fused_operands(x, Wq, sw, bias)
+    y = out if out is not None else torch.empty(M, N, dtype=torch.bfloat16, device=x.device)
+    _need_rows(y, torch.bfloat16, M, N, "out", x.device)
+    if N % 2 != 0:
+        raise ValueError("N must be even")
+    xq = xq_next if xq_next is not None else torch.empty(M, N // 2, dtype=torch.int8, device=x.device)
+    sx = sx_next if sx_next is not None else torch.empty(M, dtype=torch.float32, device=x.device)
+    _need_out(xq, torch.int8, (M, N // 2), "xq_next", x.device)
+    _need_out(sx, torch.float32, (M,), "sx_next", x.device)
+    nbytes = lib.w4a4_fused_requant_workspace_bytes(M, N, K)
+    ws = workspace(nbytes, x.device, "fused_requant") if nbytes else None
+    _check(lib.w4a4_linear_fused_requant(_ptr(x), x.stride(0), _ptr(Wq), _ptr(sw), _ptr(bias), _ptr(y), y.stride(0),
+                                         M, N, K, g, act, g_next, _ptr(xq), _ptr(sx), _ptr(ws), nbytes, _stream(x)),
+           "w4a4_linear_fused_requant")
+    return y, xq, sx
 
 
 def linear_fused_lora(x, Wq, sw, bias, A, B, scale, g=128, out=None):

@@ -190,7 +190,7 @@ int check_gemm_shape(int64_t M, int64_t N, int64_t K) {
 // weight-streaming kernel on the CUDA cores.
 int run_linear(const int8_t* Xq, const float* sx, const int8_t* Wq, const float* sw, const uint16_t* bias, void* out,
                int64_t M, int64_t N, int64_t K, int64_t ldo, int out_s32, int path, cudaStream_t stream,
-               int early_w = 0) {
+               int early_w = 0, int chain_g = 0, unsigned int* chain_amax = nullptr) {
   DeviceInfo* dev = nullptr;
   int st = current_device(&dev);
   if (st != W4A4_OK) return st;
@@ -261,6 +261,10 @@ int run_linear(const int8_t* Xq, const float* sx, const int8_t* Wq, const float*
   a.out_s32 = out_s32;
   a.status = dev->status;
   a.wait_ns = wait_limit_ns();
+  a.chain_g = chain_g;
+  a.chain_amax = chain_amax;
+  a.gelu_tab = nullptr;
+  if (chain_g != 0 && gelu_table_device(&a.gelu_tab) != cudaSuccess) return W4A4_ERR_CUDA;
   return gemm_tc_launch(tmA, tmB, tmY, a, dev->num_sms, stream) == cudaSuccess ? W4A4_OK : W4A4_ERR_CUDA;
 }
 
@@ -457,6 +461,49 @@ int w4a4_linear_fused(const uint16_t* x, int64_t ldx, const int8_t* Wq, const fl
   // whatever wrote the weights is complete when the GEMM kernel starts: the
   // weight-streaming kernels may begin reading them before their own wait.
   return run_linear(xq, sx, Wq, sw, bias, y, M, N, K, ldy, 0, path, s, 1);
+}
+
+// [packed x][sx][the next layer's row amax (fp32 bits)]
+size_t w4a4_fused_requant_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  if (M <= 0 || N <= 0 || K <= 0) return 0;
+  return w4a4_fused_workspace_bytes(M, N, K) + round256(static_cast<size_t>(M) * 4);
+}
+
+int w4a4_linear_fused_requant(const uint16_t* x, int64_t ldx, const int8_t* Wq, const float* sw, const uint16_t* bias,
+                              uint16_t* y, int64_t ldy, int64_t M, int64_t N, int64_t K, int g, int act, int g_next,
+                              int8_t* Xq_next, float* sx_next, void* workspace, size_t workspace_bytes, void* stream) {
+  int st = validate_fused(x, ldx, Wq, sw, bias, y, ldy, M, N, K, g, act);
+  if (st != W4A4_OK) return st;
+  if ((st = check_quant_shape(N, g_next)) != W4A4_OK) return st;   // N is the next layer's K
+  if (Xq_next == nullptr || sx_next == nullptr) return W4A4_ERR_NULL;
+  if (!aligned(Xq_next, 16) || !aligned(sx_next, 4)) return W4A4_ERR_ALIGN;
+  DeviceInfo* dev = nullptr;
+  if ((st = current_device(&dev)) != W4A4_OK) return st;
+  if (M == 0) return W4A4_OK;
+  const size_t need = w4a4_fused_requant_workspace_bytes(M, N, K);
+  if (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 256)) return W4A4_ERR_WORKSPACE;
+  // Layout: [packed x][sx][amax]
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int8_t* xq = reinterpret_cast<int8_t*>(ws);
+  float* sx = reinterpret_cast<float*>(ws + fused_codes_bytes(M, K));
+  unsigned int* amax = reinterpret_cast<unsigned int*>(ws + w4a4_fused_workspace_bytes(M, N, K));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int path = linear_path(M, K);
+  if (path != 0) {
+    // the weight-streaming kernels of small batches have no requantising
+    // epilogue: the layer, then the one-pass activation kernel on its output
+    if ((st = w4a4_quantize_activation(x, M, K, ldx, g, act, xq, sx, stream)) != W4A4_OK) return st;
+    if ((st = run_linear(xq, sx, Wq, sw, bias, y, M, N, K, ldy, 0, path, s, 1)) != W4A4_OK) return st;
+    return w4a4_quantize_activation(y, M, N, ldy, g_next, 1, Xq_next, sx_next, stream);
+  }
+  // the amax slots start at zero (atomic maxima of non-negative values); set
+  // before the activation kernel so that it and the GEMM stay back to back
+  if (cudaMemsetAsync(amax, 0, static_cast<size_t>(M) * 4, s) != cudaSuccess) return W4A4_ERR_CUDA;
+  if ((st = w4a4_quantize_activation(x, M, K, ldx, g, act, xq, sx, stream)) != W4A4_OK) return st;
+  if ((st = run_linear(xq, sx, Wq, sw, bias, y, M, N, K, ldy, 0, 0, s, 1, g_next, amax)) != W4A4_OK) return st;
+  return requant_bf16(y, M, static_cast<int>(N), ldy, g_next, amax, Xq_next, sx_next, dev->num_sms, s) == cudaSuccess
+             ? W4A4_OK
+             : W4A4_ERR_CUDA;
 }
 
 // [t: M x 64 bf16][the K slices' partial sums: slices x M x 64 fp32]

@@ -45,6 +45,7 @@
 
 #include <cstdint>
 
+#include "gelu_table.cuh"
 #include "ptx.cuh"
 #include "w4a4_internal.h"
 
@@ -91,9 +92,17 @@ constexpr uint32_t kOffPack = SWD * kStage;
 // epilogue staging: per epilogue warp two 32 x 32 bf16 boxes (64-byte rows,
 // 64-byte swizzle) for the TMA stores of y
 constexpr uint32_t kStageBox = 32 * 64;
-constexpr uint32_t kOffEpi = kOffPack + SP * kPStage;
-constexpr uint32_t kSmemBytes = kOffEpi + 4 * 2 * kStageBox;
-constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;   // slack for 1024-byte alignment
+// Shared-memory plan by kernel form.  The requantising epilogue (CHAIN = the
+// next layer's rotation group) keeps the GELU table in shared memory, in the
+// room of one packed stage.
+template <int CHAIN>
+struct Plan {
+  static constexpr int kSP = CHAIN ? SP - 1 : SP;   // packed ring depth
+  static constexpr uint32_t kOffEpi = kOffPack + kSP * kPStage;
+  static constexpr uint32_t kOffGelu = kOffEpi + 4 * 2 * kStageBox;
+  static constexpr uint32_t kBytes = kOffGelu + (CHAIN ? kGeluTableSize * 4 : 0);
+  static constexpr uint32_t kAlloc = kBytes + 1024;   // slack for 1024-byte alignment
+};
 
 // packed 16-byte units per CTA and k-block: (HM + HN) rows x 4 units
 constexpr int kUnits = (HM + HN) * (BKP / 16);
@@ -172,7 +181,22 @@ __device__ __forceinline__ void widen_units(const uint8_t* __restrict__ pstage, 
   }
 }
 
-template <int OUT_S32>
+// Walsh-Hadamard butterflies over 32 values in natural (Sylvester) order,
+// unnormalised.
+__device__ __forceinline__ void fwht32(uint32_t (&v)[32]) {
+#pragma unroll
+  for (int h = 1; h < 32; h <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      if (i & h) continue;
+      const float a = __uint_as_float(v[i]), b = __uint_as_float(v[i + h]);
+      v[i] = __float_as_uint(a + b);
+      v[i + h] = __float_as_uint(a - b);
+    }
+  }
+}
+
+template <int OUT_S32, int CHAIN>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmY, GemmArgs args) {
@@ -181,6 +205,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ __align__(16) float epi_sw[2][BN];
   __shared__ __align__(16) float epi_bias[2][BN];
   uint8_t* smem = align1024_shared(smem_dyn);
+  constexpr int kSP = Plan<CHAIN>::kSP;
+  float* gtab = reinterpret_cast<float*>(smem + Plan<CHAIN>::kOffGelu);   // requantising epilogue only
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -194,7 +220,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int num_kb = static_cast<int>((args.K + BK - 1) / BK);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < SP; ++s) {
+    for (int s = 0; s < kSP; ++s) {
       mbar_init(&bars.packed_full[s], 1);
       mbar_init(&bars.packed_empty[s], kWidenWarps);
     }
@@ -215,6 +241,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kWarpMma) {
     tmem_alloc_pair(&bars.tmem_base, kTmemCols);
     tmem_relinquish_pair();
+  }
+  if constexpr (CHAIN > 0) {
+    // the GELU table (filled by the host before any launch)
+    for (int i = threadIdx.x; i < kGeluTableSize; i += kThreads) gtab[i] = args.gelu_tab[i];
   }
   tc_fence_before();
   cluster_sync();   // barriers and tensor memory of both CTAs are ready
@@ -256,6 +286,47 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!OUT_S32 && mrow) sxm = args.sx[m];
     const uint64_t sx2 = pk2(sxm, sxm);
     const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + ab * BN;
+    // requantising epilogue: the largest |butterfly sum| of this row over the
+    // tile's rotation groups
+    float chain_amax_u = 0.0f;
+    // After the butterflies inside each of a group's 32-column chunks (stored
+    // back over the accumulator), the butterflies across its CHAIN / 32
+    // chunks at every position; returns the group's largest |sum|.  H_g in
+    // natural order is H_(g/32) on the chunk index times H_32 on the position.
+    auto group_cross = [&](int c0) -> float {
+      constexpr int NC = CHAIN > 0 ? CHAIN / 32 : 1;
+      constexpr int PB = NC <= 4 ? 8 : 4;   // positions per pass
+      float mx = 0.0f;
+#pragma unroll 1
+      for (int j = 0; j < 32; j += PB) {
+        uint32_t v[NC][PB];
+#pragma unroll
+        for (int cc = 0; cc < NC; ++cc) {
+          if constexpr (PB == 8) tmem_ld_32x32b_x8(tbase + (c0 + cc) * 32 + j, v[cc]);
+          else tmem_ld_32x32b_x4(tbase + (c0 + cc) * 32 + j, v[cc]);
+        }
+        tmem_wait_ld();
+#pragma unroll
+        for (int pp = 0; pp < PB; ++pp) {
+          float a[NC];
+#pragma unroll
+          for (int cc = 0; cc < NC; ++cc) a[cc] = __uint_as_float(v[cc][pp]);
+#pragma unroll
+          for (int h = 1; h < NC; h <<= 1) {
+#pragma unroll
+            for (int cc = 0; cc < NC; ++cc) {
+              if (cc & h) continue;
+              const float x0 = a[cc], x1 = a[cc + h];
+              a[cc] = x0 + x1;
+              a[cc + h] = x0 - x1;
+            }
+          }
+#pragma unroll
+          for (int cc = 0; cc < NC; ++cc) mx = fmaxf(mx, fabsf(a[cc]));
+        }
+      }
+      return mx;
+    };
     // one chunk: its tensor-memory load (issued one chunk earlier) is waited
     // for, the next chunk's load is issued into the other buffer so that it
     // overlaps this chunk's math, and the chunk is converted and stored
@@ -320,6 +391,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_store_2d(&tmY, box, static_cast<int32_t>(n0), static_cast<int32_t>(m));
         bulk_commit_group();
       }
+      if constexpr (CHAIN > 0) {
+        // the next layer's input: GELU of the bf16 outputs just stored, then
+        // the rotation's butterflies inside the chunk, written back over the
+        // chunk's accumulator columns (nothing reads them after this tile)
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          // GELU = t * Phi(t), Phi from the table, as the activation kernel forms it
+          float p0, p1;
+          gelu_phi_word(packed[i], gtab, p0, p1);
+          cur[2 * i] = __float_as_uint(__fmul_rn(__uint_as_float(packed[i] << 16), p0));
+          cur[2 * i + 1] = __float_as_uint(__fmul_rn(__uint_as_float(packed[i] & 0xFFFF0000u), p1));
+        }
+        fwht32(cur);
+        tmem_st_32x32b_x32(tbase + c * 32, cur);
+        if ((c + 1) % (CHAIN / 32) == 0) {
+          tmem_wait_st();
+          chain_amax_u = fmaxf(chain_amax_u, group_cross(c + 1 - CHAIN / 32));
+        }
+      }
     };
     // chunk ranges start on an even chunk and hold an even number of them:
     // even chunks use buffer r0, odd ones r1 (static register indexing)
@@ -328,6 +418,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int c = c_begin; c < c_end; c += 2) {
       chunk(c, r0, r1);
       chunk(c + 1, r1, r0);
+    }
+    if constexpr (CHAIN > 0) {
+      // the row's amax over this tile's groups, as fp32 bits (non-negative
+      // floats order like their bit patterns); 1/sqrt(g) applied once
+      // (rounding is monotonic, so max fl(|u| / sqrt g) = fl(max |u| / sqrt g))
+      constexpr float kNorm = CHAIN == 64 ? 0.125f : (CHAIN == 256 ? 0.0625f : 0.0883883476483184405f);
+      if (mrow) atomicMax(args.chain_amax + m, __float_as_uint(chain_amax_u * kNorm));
     }
   };
 
@@ -398,7 +495,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_2d(dst, &tmA, &bars.packed_full[ps], kb * BKP, mb * BM + static_cast<int>(rank) * HM);
           tma_load_2d(dst + kPackA, &tmB, &bars.packed_full[ps], kb * BKP, nb * BN + static_cast<int>(rank) * HN);
           ++issued;
-          if (++ps == SP) { ps = 0; ph ^= 1; }
+          if (++ps == kSP) { ps = 0; ph ^= 1; }
         }
       }
       {
@@ -406,8 +503,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // after an abort some may never be consumed, and an abort raised by
         // another role after this loop ended would otherwise go unnoticed here.
         // In a normal run every phase waited for has completed already.
-        for (int s2 = 0; s2 < SP && s2 < issued; ++s2) {
-          const int64_t n_s = issued / SP + (s2 < issued % SP ? 1 : 0);
+        for (int s2 = 0; s2 < kSP && s2 < issued; ++s2) {
+          const int64_t n_s = issued / kSP + (s2 < issued % kSP ? 1 : 0);
           (void)mbar_wait(&bars.packed_full[s2], static_cast<uint32_t>((n_s - 1) & 1), nullptr, nullptr, 100000000ull);
         }
       }
@@ -422,7 +519,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = cluster; t < tiles && ok; t += nclusters) {
       for (int kb = 0; kb < num_kb; ++kb, ++gk) {
         if (static_cast<int>(gk % kWGroups) != grp) {
-          if (++ps == SP) { ps = 0; ph ^= 1; }
+          if (++ps == kSP) { ps = 0; ph ^= 1; }
           if (++ws == SWD) { ws = 0; wph ^= 1; }
           continue;
         }
@@ -435,7 +532,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive(&bars.wide_full[ws]);
           mbar_arrive(&bars.packed_empty[ps]);
         }
-        if (++ps == SP) { ps = 0; ph ^= 1; }
+        if (++ps == kSP) { ps = 0; ph ^= 1; }
         if (++ws == SWD) { ws = 0; wph ^= 1; }
       }
     }
@@ -444,7 +541,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // every tile but the cluster's last (drained by all sixteen warps below)
     const int q = warp & 3;   // TMEM lane quarter this warp may access
     const int et = q * 32 + lane;   // 0..127 across the four epilogue warps
-    uint8_t* epi_stage = smem + kOffEpi + q * 2 * kStageBox;
+    uint8_t* epi_stage = smem + Plan<CHAIN>::kOffEpi + q * 2 * kStageBox;
     uint32_t acc_ph = 0;
     int lt = 0;
     for (int t = cluster; t + nclusters < tiles; t += nclusters, ++lt) {
@@ -486,8 +583,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool aborted = bar_sync_or(2, 512, *abort_flag != 0);
     if (!aborted) {
       tc_fence_after();
-      const int part = warp >> 2;   // 0..3 within the lane quarter
-      drain_chunks(t_last, ab, 2 * part, 2 * part + 2, smem + warp * 2 * kStageBox);
+      if constexpr (CHAIN > 0) {
+        // a rotation group spans several chunks: the four epilogue warps
+        // drain the whole tile, as for the other tiles
+        if (is_epi_warp(warp)) drain_chunks(t_last, ab, 0, BN / 32, smem + Plan<CHAIN>::kOffEpi + (warp & 3) * 2 * kStageBox);
+      } else {
+        const int part = warp >> 2;   // 0..3 within the lane quarter
+        drain_chunks(t_last, ab, 2 * part, 2 * part + 2, smem + warp * 2 * kStageBox);
+      }
     }
     if (lane == 0) bulk_wait_group_read<0>();   // every store has read its staging box
   }
@@ -503,7 +606,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // Largest number of 2-CTA clusters of this kernel that can be resident at
 // once (queried once per device; the persistent grid never exceeds it).
-template <int OUT_S32>
+template <int OUT_S32, int CHAIN>
 int max_clusters(int num_sms) {
   static int cached[64] = {0};
   int dev = 0;
@@ -512,7 +615,7 @@ int max_clusters(int num_sms) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * (num_sms / 2), 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = kSmemAlloc;
+  cfg.dynamicSmemBytes = Plan<CHAIN>::kAlloc;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
@@ -521,7 +624,7 @@ int max_clusters(int num_sms) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, gemm_tc_kernel<OUT_S32>, &cfg) != cudaSuccess || n <= 0) {
+  if (cudaOccupancyMaxActiveClusters(&n, gemm_tc_kernel<OUT_S32, CHAIN>, &cfg) != cudaSuccess || n <= 0) {
     (void)cudaGetLastError();
     n = num_sms / 2;
   }
@@ -530,7 +633,7 @@ int max_clusters(int num_sms) {
   return n;
 }
 
-template <int OUT_S32>
+template <int OUT_S32, int CHAIN>
 cudaError_t launch(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmY, const GemmArgs& a,
                    int64_t tiles, int num_sms, cudaStream_t stream) {
   static bool attr_set[64] = {};
@@ -539,17 +642,17 @@ cudaError_t launch(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtenso
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!attr_set[dev]) {
-    e = cudaFuncSetAttribute(gemm_tc_kernel<OUT_S32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kSmemAlloc));
+    e = cudaFuncSetAttribute(gemm_tc_kernel<OUT_S32, CHAIN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(Plan<CHAIN>::kAlloc));
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  const int64_t cmax = max_clusters<OUT_S32>(num_sms);
+  const int64_t cmax = max_clusters<OUT_S32, CHAIN>(num_sms);
   const int grid = static_cast<int>(2 * (tiles < cmax ? tiles : cmax));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = kSmemAlloc;
+  cfg.dynamicSmemBytes = Plan<CHAIN>::kAlloc;
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -560,7 +663,7 @@ cudaError_t launch(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtenso
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<OUT_S32>, tmA, tmB, tmY, a);
+  return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<OUT_S32, CHAIN>, tmA, tmB, tmY, a);
 }
 
 }  // namespace
@@ -569,8 +672,20 @@ cudaError_t gemm_tc_launch(const CUtensorMap& tmA, const CUtensorMap& tmB, const
                            int num_sms, cudaStream_t stream) {
   const int64_t tiles = ((a.M + BM - 1) / BM) * ((a.N + BN - 1) / BN);
   if (tiles == 0) return cudaSuccess;
-  cudaError_t e =
-      a.out_s32 ? launch<1>(tmA, tmB, tmY, a, tiles, num_sms, stream) : launch<0>(tmA, tmB, tmY, a, tiles, num_sms, stream);
+  cudaError_t e;
+  if (a.out_s32) {
+    e = launch<1, 0>(tmA, tmB, tmY, a, tiles, num_sms, stream);
+  } else if (a.chain_g == 0) {
+    e = launch<0, 0>(tmA, tmB, tmY, a, tiles, num_sms, stream);
+  } else if (a.chain_g == 64) {
+    e = launch<0, 64>(tmA, tmB, tmY, a, tiles, num_sms, stream);
+  } else if (a.chain_g == 128) {
+    e = launch<0, 128>(tmA, tmB, tmY, a, tiles, num_sms, stream);
+  } else if (a.chain_g == 256) {
+    e = launch<0, 256>(tmA, tmB, tmY, a, tiles, num_sms, stream);
+  } else {
+    return cudaErrorInvalidValue;
+  }
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

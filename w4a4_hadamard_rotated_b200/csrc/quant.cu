@@ -52,20 +52,12 @@
 #include <cstring>
 #include <mutex>
 
+#include "gelu_table.cuh"
 #include "ptx.cuh"
 #include "w4a4_internal.h"
 
 namespace w4a4 {
 
-// GELU table: Phi(t), the standard normal CDF, for the bf16 values t with
-// exponent field kGeluFirstExp .. kGeluFirstExp + kGeluExps - 1
-// (2^-12 <= |t| < 8), 128 mantissas each; entry 2 d + sign holds the value
-// whose magnitude is the d-th of that range (the two signs side by side, so
-// the sign bit lands in the byte offset with one shift and mask).
-constexpr uint32_t kGeluFirstExp = 115;
-constexpr uint32_t kGeluExps = 15;
-constexpr int kGeluMags = static_cast<int>(kGeluExps * 128);   // magnitudes per sign
-constexpr int kGeluTableSize = 2 * kGeluMags;
 __device__ float g_gelu_table[kGeluTableSize];
 
 constexpr int kSlab = 64;      // elements per thread
@@ -105,29 +97,6 @@ __device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
   uint64_t r;
   asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
   return r;
-}
-
-// GELU of the two bf16 inputs held in one 32-bit word: GELU(t) = t Phi(t)
-// with Phi(t) = (1 + erf(t / sqrt 2)) / 2 read from the table (one product,
-// so within about an ulp of the exact value).  The byte offsets of both
-// entries are formed at once, one per 16-bit half (at most 8 * 1919 + 4, so
-// no half overflows): the magnitude clamped with 16-bit SIMD min/max, minus
-// the range start, times 8, plus 4 for a negative t; clamping the exponent field to the
-// table's range is the only special case: below 2^-12 the entry of 2^-12
-// stands in (Phi differs by < 1e-4, the product by < 3e-8 absolute), at or
-// above 8 the entry of 8 - 2^-5 does, which holds 1 for positive t (Phi
-// rounds to 1 there) and 0 for negative t, so GELU is t or -0 (the exact
-// |t Phi(t)| is below 7e-15 for t <= -8 + 2^-5 and falls with |t|).  `tab`
-// is the table in shared memory.
-__device__ __forceinline__ void gelu_phi_word(uint32_t w, const float* __restrict__ tab, float& phi0, float& phi1) {
-  constexpr uint32_t lo = kGeluFirstExp << 7, hi = ((kGeluFirstExp + kGeluExps) << 7) - 1u;
-  uint32_t c;
-  asm("max.u16x2 %0, %1, %2;" : "=r"(c) : "r"(w & 0x7FFF7FFFu), "r"(lo * 0x10001u));
-  asm("min.u16x2 %0, %0, %1;" : "+r"(c) : "r"(hi * 0x10001u));
-  const uint32_t off = ((c - lo * 0x10001u) << 3) | ((w >> 13) & 0x00040004u);
-  const char* tb = reinterpret_cast<const char*>(tab);
-  phi0 = *reinterpret_cast<const float*>(tb + (off & 0xFFFFu));
-  phi1 = *reinterpret_cast<const float*>(tb + (off >> 16));
 }
 
 // bf16 bits of element e of a 16-byte chunk.
@@ -602,6 +571,153 @@ cudaError_t rotate_quant_bf16(const uint16_t* x, int64_t M, int K, int64_t ldx, 
 cudaError_t rotate_quant_f32(const float* x, int64_t M, int K, int64_t ldx, int g, int8_t* out, float* scale,
                              int num_sms, unsigned int* status, cudaStream_t stream) {
   return dispatch_rq<float>(x, M, K, ldx, g, 0, out, scale, num_sms, status, stream);
+}
+
+// ---- Second pass of a requantising GEMM epilogue: GELU, rotation and
+// quantisation of a layer's bf16 output with the row amax already known
+// (the GEMM's epilogue reported it), so no row reduction and no barrier.
+// Thread = one 64-element slab, loaded straight from global memory (eight
+// 16-byte loads); a warp takes 32 consecutive slabs of the row-major [M, K]
+// slab grid, so a rotation group (g / 64 slabs) sits in lanes l, l ^ 1
+// (and l ^ 2) of one warp.  The arithmetic is the register quantiser's: the
+// GELU table, f32x2 butterflies, one shuffle stage per 64 elements beyond 64,
+// codes by one fused multiply-add with the magic number and a Horner chain.
+constexpr int kRqThreads = 128;
+constexpr int kRqCtasPerSm = 5;
+
+template <int G>
+__global__ void __launch_bounds__(kRqThreads, kRqCtasPerSm)
+    requant_kernel(const uint16_t* __restrict__ y, int64_t M, int K, int64_t ldy,
+                   const unsigned int* __restrict__ amax_bits, int8_t* __restrict__ out, float* __restrict__ scale) {
+  __shared__ float gelu_tab[kGeluTableSize];
+  for (int i = threadIdx.x; i < kGeluTableSize; i += blockDim.x) gelu_tab[i] = g_gelu_table[i];
+  // y and the row amax come from the GEMM launched before this kernel
+  griddep_wait();
+  griddep_launch_dependents();
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int S = K / kSlab;
+  const int64_t total = M * S;
+  const float norm = G == 64 ? 0.125f : (G == 256 ? 0.0625f : 0.0883883476483184405f);
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (kRqThreads / 32);
+  const uint64_t magic2 = pk2(kMagic8, kMagic8);
+  for (int64_t base = (static_cast<int64_t>(blockIdx.x) * (kRqThreads / 32) + (threadIdx.x >> 5)) * 32; base < total;
+       base += warps * 32) {
+    const int64_t slab = base + lane;
+    const bool valid = slab < total;   // whole rotation groups are valid or not (S % (G / 64) == 0)
+    const int64_t row = valid ? slab / S : 0;
+    const int s = valid ? static_cast<int>(slab - row * S) : 0;
+    uint64_t V[kHalf];
+    {
+      const uint16_t* src = y + row * ldy + static_cast<int64_t>(s) * kSlab;
+      uint4 ch[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        ch[j] = valid ? *reinterpret_cast<const uint4*>(src + 8 * j) : make_uint4(0u, 0u, 0u, 0u);
+      // V[i] = (element i, element i + 32): chunk j < 4 gives the low halves
+      // of V[8j .. 8j+7], chunk j + 4 the high halves
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint4 lo = ch[j], hi = ch[j + 4];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          V[8 * j + e] = pk2(elem(lo, e, y), elem(hi, e, y));
+          if (e & 1) {
+            float pa0, pa1, pb0, pb1;
+            gelu_phi_word(bits16(lo, e - 1) | (bits16(lo, e) << 16), gelu_tab, pa0, pa1);
+            gelu_phi_word(bits16(hi, e - 1) | (bits16(hi, e) << 16), gelu_tab, pb0, pb1);
+            V[8 * j + e - 1] = mul2(V[8 * j + e - 1], pk2(pa0, pb0));
+            V[8 * j + e] = mul2(V[8 * j + e], pk2(pa1, pb1));
+          }
+        }
+      }
+    }
+    fht_stage2<1>(V);
+    fht_stage2<2>(V);
+    fht_stage2<4>(V);
+    fht_stage2<8>(V);
+    fht_stage2<16>(V);
+#pragma unroll
+    for (int i = 0; i < kHalf; ++i) {
+      float a, b;
+      upk2(V[i], a, b);
+      V[i] = pk2(a + b, a - b);
+    }
+    // across slabs: the lower slab of a pair keeps a + b, the upper one a - b
+    if (G >= 128) {
+      const float sg = (s & 1) ? -1.0f : 1.0f;
+      const uint64_t sg2 = pk2(sg, sg);
+#pragma unroll
+      for (int i = 0; i < kHalf; ++i) V[i] = fma2(V[i], sg2, __shfl_xor_sync(0xFFFFFFFFu, V[i], 1));
+    }
+    if (G == 256) {
+      const float sg = (s & 2) ? -1.0f : 1.0f;
+      const uint64_t sg2 = pk2(sg, sg);
+#pragma unroll
+      for (int i = 0; i < kHalf; ++i) V[i] = fma2(V[i], sg2, __shfl_xor_sync(0xFFFFFFFFu, V[i], 2));
+    }
+    if (!valid) continue;
+    const float amax_r = __uint_as_float(amax_bits[row]);
+    const float sc = amax_r / 7.0f;   // fp32 division, as the method states
+    if (s == 0) scale[row] = sc;
+    const float ni = sc > 0.0f ? norm * (1.0f / sc) : 0.0f;
+    const uint64_t mult = pk2(ni, ni);
+    uint32_t packed[kSlab / 8];
+#pragma unroll
+    for (int w = 0; w < kHalf / 8; ++w) {
+      uint32_t lo_acc = 0u, hi_acc = 0u;
+#pragma unroll
+      for (int e = 7; e >= 0; --e) {
+        const uint64_t f = fma2(V[8 * w + e], mult, magic2);
+        float f0, f1;
+        upk2(f, f0, f1);
+        lo_acc = lo_acc * 16u + __float_as_uint(f0);
+        hi_acc = hi_acc * 16u + __float_as_uint(f1);
+      }
+      packed[w] = (lo_acc - kHornerBias) ^ 0x88888888u;
+      packed[w + kHalf / 8] = (hi_acc - kHornerBias) ^ 0x88888888u;
+    }
+    uint4* dst = reinterpret_cast<uint4*>(out + row * static_cast<int64_t>(K / 2) + static_cast<int64_t>(s) * (kSlab / 2));
+    dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+    dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+  }
+}
+
+cudaError_t gelu_table_device(const float** table) {
+  const cudaError_t e = ensure_gelu_table();
+  if (e != cudaSuccess) return e;
+  void* p = nullptr;
+  const cudaError_t e2 = cudaGetSymbolAddress(&p, g_gelu_table);
+  if (e2 != cudaSuccess) return e2;
+  *table = static_cast<const float*>(p);
+  return cudaSuccess;
+}
+
+cudaError_t requant_bf16(const uint16_t* y, int64_t M, int K, int64_t ldy, int g, const unsigned int* amax,
+                         int8_t* out, float* scale, int num_sms, cudaStream_t stream) {
+  if (M == 0) return cudaSuccess;
+  const cudaError_t e = ensure_gelu_table();
+  if (e != cudaSuccess) return e;
+  const int64_t warps_needed = (M * (K / kSlab) + 31) / 32;
+  int64_t ctas = static_cast<int64_t>(num_sms) * kRqCtasPerSm;
+  const int64_t need = (warps_needed + kRqThreads / 32 - 1) / (kRqThreads / 32);
+  if (ctas > need) ctas = need;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(ctas), 1, 1);
+  cfg.blockDim = dim3(kRqThreads, 1, 1);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t r;
+  if (g == 64) r = cudaLaunchKernelEx(&cfg, requant_kernel<64>, y, M, K, ldy, amax, out, scale);
+  else if (g == 128) r = cudaLaunchKernelEx(&cfg, requant_kernel<128>, y, M, K, ldy, amax, out, scale);
+  else if (g == 256) r = cudaLaunchKernelEx(&cfg, requant_kernel<256>, y, M, K, ldy, amax, out, scale);
+  else return cudaErrorInvalidValue;
+  if (r != cudaSuccess) return r;
+  return cudaGetLastError();
 }
 
 }  // namespace w4a4

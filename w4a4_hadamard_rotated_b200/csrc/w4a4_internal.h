@@ -40,6 +40,15 @@ cudaError_t rotate_quant_bf16(const uint16_t* x, int64_t M, int K, int64_t ldx, 
                               float* scale, int num_sms, unsigned int* status, cudaStream_t stream, int path = 0);
 // Which kernel path 0 picks: 1 (register butterflies) or 2 (tensor cores).
 int rotate_quant_bf16_route(int64_t M, int K, int g, int act);
+// Codes and row scales of GELU(y) for the next layer, rotation group g, from
+// a bf16 y [M, K] (row stride ldy, 16-byte aligned rows) and the row amax of
+// the rotated values as fp32 bits (amax [M], from the GEMM's requantising
+// epilogue).  K % g == 0, K % 128 == 0.
+// Device address of the GELU table (gelu_table.cuh), filled on first use;
+// the first call on a device must not be inside a stream capture.
+cudaError_t gelu_table_device(const float** table);
+cudaError_t requant_bf16(const uint16_t* y, int64_t M, int K, int64_t ldy, int g, const unsigned int* amax,
+                         int8_t* out, float* scale, int num_sms, cudaStream_t stream);
 cudaError_t rotate_quant_f32(const float* x, int64_t M, int K, int64_t ldx, int g, int8_t* out, float* scale,
                              int num_sms, unsigned int* status, cudaStream_t stream);
 // Tensor-core form of rotate_quant_bf16 for act = 0, g in {64, 128} and
@@ -63,6 +72,13 @@ struct GemmArgs {
   int out_s32;            // 1: raw int32 accumulators
   unsigned int* status;   // device status word (bounded-wait timeouts)
   unsigned long long wait_ns;   // bounded-wait limit (wait_limit_ns())
+  // Requantising epilogue for a following layer (0: off; else its rotation
+  // group 64, 128 or 256): per row, atomicMax of fp32 bits of the amax of
+  // rotate(GELU(y)) over each tile's columns into chain_amax [M] (zeroed
+  // before the launch).
+  int chain_g;
+  unsigned int* chain_amax;
+  const float* gelu_tab;   // the GELU table in device memory (gelu_table_device)
 };
 // tmA: packed activations [M, K/2] bytes, tmB: packed weights [N, K/2] bytes,
 // both with box {64 bytes, kGemmBM/2 rows}; tmY: bf16 output [M, N] (row
