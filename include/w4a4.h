@@ -234,6 +234,8 @@ int w4a4_linear_fused_noalloc(const uint16_t* x, int64_t ldx, const int8_t* Wq, 
  *   workspace: w4a4_fused_requant_workspace_bytes(M, N, K) bytes, 256-byte
  *       aligned (the activation codes of x, their scales and the row amax
  *       slots; the call sets the slots to zero itself).
+ *   The first call on a device uploads the GELU table as w4a4_quantize_
+ *   activation with act = 1 does: make it before any stream capture.
  * y is bit-identical to w4a4_linear_fused's.  Xq_next and sx_next match the
  * one-pass activation kernel up to the rounding of the rotated values (both
  * passes form GELU with its table; the rotation is summed in another order).
