@@ -111,3 +111,24 @@ def test_requant_small_batch_uses_the_one_pass_kernel(cuda_lib):
     y, xq, sx = cuda_lib.linear_fused_requant(x.cuda(), Wq, sw, b.cuda(), 128, 0, 128)
     xq1, sx1 = cuda_lib.quantize_activation(y, 128, 1)
     assert torch.equal(xq, xq1) and torch.equal(sx, sx1)
+
+
+def test_requant_epilogue_gelu_input_and_strided_output(cuda_lib):
+    """A chain link inside a chain: a GELU input (act = 1, g = 64) and y
+    written into a column slice of a wider buffer (row stride N + 64); the
+    padding columns keep their values and the codes still match the oracle."""
+    M, K, N, g, g_next = 257, 512, 640, 64, 128
+    cfg = workloads.Linear("chain gelu", M=M, K=K, N=N, g=g, seed=41, act=1)
+    x, W, b = cfg.make()
+    xc = x.cuda()
+    Wq, sw = cuda_lib.quantize_weight(W.cuda(), g)
+    wide = workloads.make_activation(M, N + 64, seed=42).cuda()
+    pad = wide[:, N:].clone()
+    y, xq, sx = cuda_lib.linear_fused_requant(xc, Wq, sw, b.cuda(), g, 1, g_next, out=wide[:, :N])
+    assert torch.equal(wide[:, N:].view(torch.int16), pad.view(torch.int16))
+    y_plain = cuda_lib.linear_fused(xc, Wq, sw, b.cuda(), g, 1)
+    assert torch.equal(y.contiguous().view(torch.int16), y_plain.view(torch.int16))
+    ref = orc.chain_requant(to_np_bits(y.cpu()), g_next, BLOCK, act=1)
+    _chain_scale_ok(sx.cpu().numpy(), ref["scale"], g_next)
+    check_packed(xq.cpu(), torch.from_numpy(ref["scale"]), ref, "chain gelu strided", g_next)
+    assert cuda_lib.last_device_error() == 0

@@ -413,7 +413,7 @@ def test_bounded_wait_reports_timeout_and_context_survives(cuda_lib):
 
 
 @pytest.mark.parametrize("kernel", ["quant_butterfly", "quant_tensor_core", "gemm_tc", "gemm_small_m",
-                                    "fused_square", "lora"])
+                                    "fused_square", "lora", "requant_chain"])
 def test_product_kernel_waits_expire_and_context_survives(cuda_lib, kernel):
     """With a wait limit of a few nanoseconds the product kernels' waits on
     their copy rings, widened stages, accumulators and cluster peers expire
@@ -443,6 +443,9 @@ def test_product_kernel_waits_expire_and_context_survives(cuda_lib, kernel):
         "gemm_small_m": lambda: cuda_lib.linear(Xq16, sx16, Wqk, swk),
         "fused_square": lambda: cuda_lib.linear_fused(big, Wq, sw, None, g),
         "lora": lambda: cuda_lib.lora_add(big, A, B, 0.25, ylora),
+        # the GEMM instance with the requantising epilogue (its second pass
+        # has no waits and runs on whatever the aborted GEMM left)
+        "requant_chain": lambda: cuda_lib.linear_fused_requant(big, Wq, sw, None, g, 0, 128),
     }
     if kernel == "gemm_small_m":
         assert cuda_lib.linear_kernel(16, 3072, 12288) == 1

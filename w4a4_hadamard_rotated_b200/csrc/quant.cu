@@ -576,62 +576,97 @@ cudaError_t rotate_quant_f32(const float* x, int64_t M, int K, int64_t ldx, int 
 // ---- Second pass of a requantising GEMM epilogue: GELU, rotation and
 // quantisation of a layer's bf16 output with the row amax already known
 // (the GEMM's epilogue reported it), so no row reduction and no barrier.
-// Thread = one 64-element slab, loaded straight from global memory (eight
-// 16-byte loads); a warp takes 32 consecutive slabs of the row-major [M, K]
-// slab grid, so a rotation group (g / 64 slabs) sits in lanes l, l ^ 1
-// (and l ^ 2) of one warp.  The arithmetic is the register quantiser's: the
-// GELU table, f32x2 butterflies, one shuffle stage per 64 elements beyond 64,
+// Thread = one 64-element slab; a warp takes 32 consecutive slabs of the
+// row-major [M, K] slab grid, so a rotation group (g / 64 slabs) sits in
+// lanes l, l ^ 1 (and l ^ 2) of one warp.  Each warp streams its slabs
+// through a two-stage ring of its own in shared memory with 16-byte
+// cp.async copies (the next block of 32 slabs is in flight while the warp
+// computes the current one; a lane's slab sits at lane * 128 bytes with
+// 16-byte chunk j at j ^ (lane & 7), so the copies and the reads are free of
+// bank conflicts).  The arithmetic is the register quantiser's: the GELU
+// table, f32x2 butterflies, one shuffle stage per 64 elements beyond 64,
 // codes by one fused multiply-add with the magic number and a Horner chain.
 constexpr int kRqThreads = 128;
-constexpr int kRqCtasPerSm = 5;
+constexpr int kRqCtasPerSm = 4;
+constexpr int kRqStages = 2;
+constexpr int kRqStageBytes = 32 * kSlab * 2;   // 4 KB: one warp's 32 slabs
+constexpr int kRqSmem = kGeluTableSize * 4 + (kRqThreads / 32) * kRqStages * kRqStageBytes;
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
 
 template <int G>
 __global__ void __launch_bounds__(kRqThreads, kRqCtasPerSm)
     requant_kernel(const uint16_t* __restrict__ y, int64_t M, int K, int64_t ldy,
                    const unsigned int* __restrict__ amax_bits, int8_t* __restrict__ out, float* __restrict__ scale) {
-  __shared__ float gelu_tab[kGeluTableSize];
+  extern __shared__ __align__(128) uint8_t rq_smem[];
+  float* gelu_tab = reinterpret_cast<float*>(rq_smem);
   for (int i = threadIdx.x; i < kGeluTableSize; i += blockDim.x) gelu_tab[i] = g_gelu_table[i];
-  // y and the row amax come from the GEMM launched before this kernel
-  griddep_wait();
-  griddep_launch_dependents();
-  __syncthreads();
   const int lane = threadIdx.x & 31;
+  const int wib = threadIdx.x >> 5;
+  const uint32_t ring = smem_u32(rq_smem + kGeluTableSize * 4 + wib * kRqStages * kRqStageBytes) + lane * (kSlab * 2);
+  const int L = lane & 7;
   const int S = K / kSlab;
   const int64_t total = M * S;
   const float norm = G == 64 ? 0.125f : (G == 256 ? 0.0625f : 0.0883883476483184405f);
   const int64_t warps = static_cast<int64_t>(gridDim.x) * (kRqThreads / 32);
   const uint64_t magic2 = pk2(kMagic8, kMagic8);
-  for (int64_t base = (static_cast<int64_t>(blockIdx.x) * (kRqThreads / 32) + (threadIdx.x >> 5)) * 32; base < total;
-       base += warps * 32) {
+  // y and the row amax come from the GEMM launched before this kernel
+  griddep_wait();
+  griddep_launch_dependents();
+  __syncthreads();
+
+  // copies of the slab block at `b` into ring stage `st` (lanes past the end
+  // copy nothing; their stage contents are never used)
+  auto fetch = [&](int64_t b, int st) {
+    const int64_t sl = b + lane;
+    if (sl < total) {
+      const int64_t r = sl / S;
+      const uint16_t* src = y + r * ldy + (sl - r * S) * kSlab;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) cp_async16(ring + st * kRqStageBytes + ((j ^ L) << 4), src + 8 * j);
+    }
+    cp_async_commit();
+  };
+  int64_t base = (static_cast<int64_t>(blockIdx.x) * (kRqThreads / 32) + wib) * 32;
+#pragma unroll
+  for (int k = 0; k < kRqStages - 1; ++k) fetch(base + k * warps * 32, k);   // empty groups past the end
+  for (int it = 0; base < total; base += warps * 32, ++it) {
+    const int st = it % kRqStages;
+    fetch(base + (kRqStages - 1) * warps * 32, (it + kRqStages - 1) % kRqStages);
+    cp_async_wait<kRqStages - 1>();      // this stage's copies have landed
+    __syncwarp();
     const int64_t slab = base + lane;
     const bool valid = slab < total;   // whole rotation groups are valid or not (S % (G / 64) == 0)
     const int64_t row = valid ? slab / S : 0;
     const int s = valid ? static_cast<int>(slab - row * S) : 0;
     uint64_t V[kHalf];
-    {
-      const uint16_t* src = y + row * ldy + static_cast<int64_t>(s) * kSlab;
-      uint4 ch[8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j)
-        ch[j] = valid ? *reinterpret_cast<const uint4*>(src + 8 * j) : make_uint4(0u, 0u, 0u, 0u);
-      // V[i] = (element i, element i + 32): chunk j < 4 gives the low halves
-      // of V[8j .. 8j+7], chunk j + 4 the high halves
+    for (int j = 0; j < 4; ++j) {
+      // V[i] = (element i, element i + 32): chunk j gives the low halves of
+      // V[8j .. 8j+7], chunk j + 4 the high halves
+      const uint4 lo = lds128(ring + st * kRqStageBytes + ((j ^ L) << 4));
+      const uint4 hi = lds128(ring + st * kRqStageBytes + (((j + 4) ^ L) << 4));
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const uint4 lo = ch[j], hi = ch[j + 4];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          V[8 * j + e] = pk2(elem(lo, e, y), elem(hi, e, y));
-          if (e & 1) {
-            float pa0, pa1, pb0, pb1;
-            gelu_phi_word(bits16(lo, e - 1) | (bits16(lo, e) << 16), gelu_tab, pa0, pa1);
-            gelu_phi_word(bits16(hi, e - 1) | (bits16(hi, e) << 16), gelu_tab, pb0, pb1);
-            V[8 * j + e - 1] = mul2(V[8 * j + e - 1], pk2(pa0, pb0));
-            V[8 * j + e] = mul2(V[8 * j + e], pk2(pa1, pb1));
-          }
+      for (int e = 0; e < 8; ++e) {
+        V[8 * j + e] = pk2(elem(lo, e, y), elem(hi, e, y));
+        if (e & 1) {
+          float pa0, pa1, pb0, pb1;
+          gelu_phi_word(bits16(lo, e - 1) | (bits16(lo, e) << 16), gelu_tab, pa0, pa1);
+          gelu_phi_word(bits16(hi, e - 1) | (bits16(hi, e) << 16), gelu_tab, pb0, pb1);
+          V[8 * j + e - 1] = mul2(V[8 * j + e - 1], pk2(pa0, pb0));
+          V[8 * j + e] = mul2(V[8 * j + e], pk2(pa1, pb1));
         }
       }
     }
+    // every lane has read this stage: the next fetch may overwrite it
+    __syncwarp();
     fht_stage2<1>(V);
     fht_stage2<2>(V);
     fht_stage2<4>(V);
@@ -681,6 +716,7 @@ __global__ void __launch_bounds__(kRqThreads, kRqCtasPerSm)
     dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
     dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
   }
+  cp_async_wait<0>();   // no copy outlives the CTA
 }
 
 cudaError_t gelu_table_device(const float** table) {
@@ -702,9 +738,22 @@ cudaError_t requant_bf16(const uint16_t* y, int64_t M, int K, int64_t ldy, int g
   int64_t ctas = static_cast<int64_t>(num_sms) * kRqCtasPerSm;
   const int64_t need = (warps_needed + kRqThreads / 32 - 1) / (kRqThreads / 32);
   if (ctas > need) ctas = need;
+  static bool attr_set[64][3] = {};
+  int dev = 0;
+  cudaError_t ea = cudaGetDevice(&dev);
+  if (ea != cudaSuccess) return ea;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  const int gi = g == 64 ? 0 : (g == 128 ? 1 : 2);
+  if (!attr_set[dev][gi]) {
+    ea = cudaFuncSetAttribute(g == 64 ? requant_kernel<64> : (g == 128 ? requant_kernel<128> : requant_kernel<256>),
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, kRqSmem);
+    if (ea != cudaSuccess) return ea;
+    attr_set[dev][gi] = true;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(ctas), 1, 1);
   cfg.blockDim = dim3(kRqThreads, 1, 1);
+  cfg.dynamicSmemBytes = kRqSmem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
