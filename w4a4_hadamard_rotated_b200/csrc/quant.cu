@@ -601,7 +601,15 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-template <int G>
+// Row and slab of slab index i over S slabs per row; 32-bit division where
+// the slab count fits (I32).
+template <bool I32>
+__device__ __forceinline__ int64_t rq_row(int64_t i, int S) {
+  if (I32) return static_cast<int64_t>(static_cast<uint32_t>(i) / static_cast<uint32_t>(S));
+  return i / S;
+}
+
+template <int G, bool I32>
 __global__ void __launch_bounds__(kRqThreads, kRqCtasPerSm)
     requant_kernel(const uint16_t* __restrict__ y, int64_t M, int K, int64_t ldy,
                    const unsigned int* __restrict__ amax_bits, int8_t* __restrict__ out, float* __restrict__ scale) {
@@ -627,7 +635,7 @@ __global__ void __launch_bounds__(kRqThreads, kRqCtasPerSm)
   auto fetch = [&](int64_t b, int st) {
     const int64_t sl = b + lane;
     if (sl < total) {
-      const int64_t r = sl / S;
+      const int64_t r = rq_row<I32>(sl, S);
       const uint16_t* src = y + r * ldy + (sl - r * S) * kSlab;
 #pragma unroll
       for (int j = 0; j < 8; ++j) cp_async16(ring + st * kRqStageBytes + ((j ^ L) << 4), src + 8 * j);
@@ -644,7 +652,7 @@ __global__ void __launch_bounds__(kRqThreads, kRqCtasPerSm)
     __syncwarp();
     const int64_t slab = base + lane;
     const bool valid = slab < total;   // whole rotation groups are valid or not (S % (G / 64) == 0)
-    const int64_t row = valid ? slab / S : 0;
+    const int64_t row = valid ? rq_row<I32>(slab, S) : 0;
     const int s = valid ? static_cast<int>(slab - row * S) : 0;
     uint64_t V[kHalf];
 #pragma unroll
@@ -738,15 +746,21 @@ cudaError_t requant_bf16(const uint16_t* y, int64_t M, int K, int64_t ldy, int g
   int64_t ctas = static_cast<int64_t>(num_sms) * kRqCtasPerSm;
   const int64_t need = (warps_needed + kRqThreads / 32 - 1) / (kRqThreads / 32);
   if (ctas > need) ctas = need;
-  static bool attr_set[64][3] = {};
+  static bool attr_set[64][6] = {};
   int dev = 0;
   cudaError_t ea = cudaGetDevice(&dev);
   if (ea != cudaSuccess) return ea;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  const int gi = g == 64 ? 0 : (g == 128 ? 1 : 2);
+  const bool i32 = M * (K / kSlab) + static_cast<int64_t>(ctas) * kRqThreads * 2 < (int64_t(1) << 31);
+  using Fn = void (*)(const uint16_t*, int64_t, int, int64_t, const unsigned int*, int8_t*, float*);
+  Fn fn = nullptr;
+  if (g == 64) fn = i32 ? requant_kernel<64, true> : requant_kernel<64, false>;
+  else if (g == 128) fn = i32 ? requant_kernel<128, true> : requant_kernel<128, false>;
+  else if (g == 256) fn = i32 ? requant_kernel<256, true> : requant_kernel<256, false>;
+  else return cudaErrorInvalidValue;
+  const int gi = (g == 64 ? 0 : (g == 128 ? 1 : 2)) * 2 + (i32 ? 1 : 0);
   if (!attr_set[dev][gi]) {
-    ea = cudaFuncSetAttribute(g == 64 ? requant_kernel<64> : (g == 128 ? requant_kernel<128> : requant_kernel<256>),
-                              cudaFuncAttributeMaxDynamicSharedMemorySize, kRqSmem);
+    ea = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kRqSmem);
     if (ea != cudaSuccess) return ea;
     attr_set[dev][gi] = true;
   }
@@ -760,11 +774,7 @@ cudaError_t requant_bf16(const uint16_t* y, int64_t M, int K, int64_t ldy, int g
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t r;
-  if (g == 64) r = cudaLaunchKernelEx(&cfg, requant_kernel<64>, y, M, K, ldy, amax, out, scale);
-  else if (g == 128) r = cudaLaunchKernelEx(&cfg, requant_kernel<128>, y, M, K, ldy, amax, out, scale);
-  else if (g == 256) r = cudaLaunchKernelEx(&cfg, requant_kernel<256>, y, M, K, ldy, amax, out, scale);
-  else return cudaErrorInvalidValue;
+  const cudaError_t r = cudaLaunchKernelEx(&cfg, fn, y, M, K, ldy, amax, out, scale);
   if (r != cudaSuccess) return r;
   return cudaGetLastError();
 }
