@@ -36,6 +36,14 @@
 //     formed with separately rounded fp32 steps (paired .f32x2 arithmetic);
 //     each 32 x 32 bf16 block is staged in shared memory (64-byte swizzle)
 //     and written with one TMA tensor store, which also clips the M/N tails.
+//   * A second instance (CHAIN = g of the next layer) adds a requantising
+//     epilogue for layer chains: after storing each 32-column chunk of y it
+//     applies GELU (t * Phi(t) from a table in shared memory, which takes the
+//     room of one packed stage) and the Walsh-Hadamard butterflies inside the
+//     chunk, writes the chunk back over its accumulator columns, and after a
+//     rotation group's last chunk runs the butterflies across the group's
+//     chunks; one atomicMax per row and tile records the largest rotated
+//     magnitude for the pass that quantises y for the next layer.
 //   * The kernel is persistent: the clusters walk the tiles with a static
 //     stride.  Every wait is bounded: an expired wait records W4A4_ERR_TIMEOUT
 //     in the device status word, every role stops, the MMAs are drained and
