@@ -135,3 +135,29 @@ def test_lora_into_a_strided_y_keeps_the_padding(cuda_lib, M, N):
     assert torch.equal(wide[:, :N].view(torch.int16), compact.view(torch.int16))
     assert torch.equal(wide[:, N:].view(torch.int16), pad0.view(torch.int16))
     assert cuda_lib.last_device_error() == 0
+
+
+def test_lora_add_with_k_not_a_multiple_of_the_chunk(cuda_lib):
+    """w4a4_lora_add accepts any K % 8 == 0: the last 64-element chunk of x
+    and A is partly past K (zero-filled by the copies).  With no rotation
+    group to speak of, the reference is the plain product the header states,
+    t = x A^T, then y += scale * t B^T, in float64."""
+    M, K, N, r = 300, 1000, 264, 48
+    x = workloads.make_activation(M, K, seed=51)
+    A, B = _lora_inputs(N, K, r, seed=52)
+    y0 = workloads.make_activation(M, N, seed=53)
+    y = y0.clone().cuda()
+    scale = 0.5
+    cuda_lib.lora_add(x.cuda(), A.cuda(), B.cuda(), scale, y)
+    xb = workloads.bf16_bits(x)
+    xf = orc.bf16_bits_to_f32(xb).astype(np.float64)
+    Af = orc.bf16_bits_to_f32(workloads.bf16_bits(A)).astype(np.float64)
+    Bf = orc.bf16_bits_to_f32(workloads.bf16_bits(B)).astype(np.float64)
+    t_ref = xf @ Af.T
+    base = orc.bf16_bits_to_f32(workloads.bf16_bits(y0)).astype(np.float64)
+    want = base + scale * (t_ref @ Bf.T)
+    got = orc.bf16_bits_to_f32(to_np_bits(y.cpu())).astype(np.float64)
+    tol = _bound(xb, A, B, scale, t_ref, want, base)
+    bad = np.abs(got - want) > tol
+    assert not bad.any(), f"{int(bad.sum())} outputs off; worst excess {np.max(np.abs(got - want) - tol):.3g}"
+    assert cuda_lib.last_device_error() == 0
